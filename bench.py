@@ -1,0 +1,348 @@
+"""Benchmark of one DSpark round (draft -> schedule -> verify) on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen3] [--impl reference]
+
+A step is one round over the qwen3-shaped workload (B=64 requests, K=8 draft
+positions, V=151,936, rank-256 bf16 Markov factors), inputs resident in HBM.
+L2 is flushed (512 MB write, untimed) before every timed round, as a target
+forward pass would between rounds; each round is timed with CUDA events on
+its stream and the per-kernel stages with events around each library call.
+Under torchrun every rank runs an independent replica (the path has no
+exchange step; weak scaling) and the time is the max over ranks.
+
+--impl reference times the CPU oracle (oracle/, fp64 numpy) on the host on a
+bounded sample of the same workload (a few requests per round, scaled to the
+full batch); it is the baseline arm, not a GPU implementation.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": HBM_FALLBACK_GBS, "source": "fallback"}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period: float = 0.1):
+        self.samples, self.reasons, self.period = [], set(), period
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def cpu_baseline(inp: dict, seconds: float = 15.0) -> dict:
+    """The oracle as it stands, on host cores, on a bounded sample of requests."""
+    import oracle
+    try:
+        import threadpoolctl
+        cores = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    B = inp["base"].shape[0]
+    n_req, rounds, spent = 4, 0, 0.0
+    t_start = time.perf_counter()
+    while spent < seconds and rounds < 64:
+        reqs = (np.arange(n_req) + rounds * n_req) % B
+        t0 = time.perf_counter()
+        oracle.run_round(inp, requests=reqs)
+        spent += time.perf_counter() - t0
+        rounds += 1
+        if time.perf_counter() - t_start > 2 * seconds:
+            break
+    sec_per_round = spent / rounds * (B / n_req)
+    return {"value": 1.0 / sec_per_round, "unit": "rounds/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{rounds} oracle rounds of {n_req} of {B} requests each (draft+verify per request, "
+                      f"schedule on the full batch), scaled by {B}/{n_req}; {spent:.1f} s of CPU work"}
+
+
+def draft_bytes(B, K, V, r, factor_bytes):
+    """Algorithmic HBM bytes of one draft launch: base read + z write + Bf once
+    + gathered A rows + per-position outputs."""
+    return B * K * V * 4 * 2 + r * V * factor_bytes + B * K * r * factor_bytes + B * K * (4 + 4 + 8 + 4)
+
+
+def verify_bytes(V, K, verify_len, accepted):
+    """Algorithmic HBM bytes of one verify call: every target row 0..L_b once,
+    plus the z row of each rejected request (the residual needs q there)."""
+    rows = int((verify_len + 1).sum())
+    rejected = int((accepted < verify_len).sum())
+    return rows * V * 4 + rejected * V * 4
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = synth.workload(args.workload)
+    inp = synth.make_round(w)
+    for _ in range(args.warmup):
+        cpu_baseline(inp, seconds=0.5)
+    t0 = time.perf_counter()
+    cb = None
+    vals = []
+    for _ in range(args.steps):
+        cb = cpu_baseline(inp, seconds=max(2.0, 20.0 / max(1, args.steps)))
+        vals.append(cb["value"])
+    value = statistics.median(vals)
+    cb["value"] = value
+    line = {"impl": "reference", "metric": "draft+schedule+verify rounds/sec", "value": value,
+            "unit": "rounds/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": config_of(w), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "rounds/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": time.perf_counter() - t0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w):
+    return {"workload": f"{w.name}: B={w.B} K={w.K} V={w.V} r={w.r} {w.factor_dtype} factors, fp32 logits",
+            "B": w.B, "K": w.K, "V": w.V, "r": w.r, "seed": w.seed,
+            "l2": "flushed by a 512 MB write before every timed round (untimed)",
+            "parallelism": "replicas (one independent round per GPU)"}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from speculative_decoding_semi_b200 import dspark_read_device_error
+    from speculative_decoding_semi_b200 import round as rnd
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = synth.workload(args.workload)
+    inp = synth.make_round(w, seed=w.seed + rank)
+    B, K, V, r = w.B, w.K, w.V, w.r
+    d = rnd.to_device(inp)
+    bufs = rnd.RoundBuffers(B, K, V, r)
+    stream = torch.cuda.Stream()
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    launches_per_round = 1 + 2 + 3  # draft, schedule (rank, final), verify (rows, decide, final)
+
+    def one_round(ev=None):
+        with torch.cuda.stream(stream):
+            flush.fill_(1.0)
+            if ev:
+                ev[0].record(stream)
+            rnd.draft(d, bufs, stream)
+            if ev:
+                ev[1].record(stream)
+            rnd.schedule(d, bufs, stream)
+            if ev:
+                ev[2].record(stream)
+            rnd.verify(d, bufs, stream=stream)
+            if ev:
+                ev[3].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        one_round()
+    torch.cuda.synchronize()
+    st, detail = dspark_read_device_error(bufs.workspace, stream)
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {detail:#x} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for k in range(args.steps):
+            one_round(evs[k])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    st, detail = dspark_read_device_error(bufs.workspace, stream)
+    if st != 0:
+        raise RuntimeError(f"device error {st} detail {detail:#x} in the timed region")
+    t_draft = [e[0].elapsed_time(e[1]) for e in evs]
+    t_sched = [e[1].elapsed_time(e[2]) for e in evs]
+    t_ver = [e[2].elapsed_time(e[3]) for e in evs]
+    t_round = [a + b + c for a, b, c in zip(t_draft, t_sched, t_ver)]
+    total_ms = sum(t_round)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    rounds_total = args.steps * world
+    value = rounds_total / (total_ms / 1000.0)
+
+    L = bufs.verify_len.cpu().numpy()
+    acc = bufs.accepted.cpu().numpy()
+    n_out = bufs.n_out.cpu().numpy()
+    peaks = measured_peaks()
+    fb = 2 if w.factor_dtype == "bf16" else 4
+    dbytes = draft_bytes(B, K, V, r, fb)
+    vbytes = verify_bytes(V, K, L, acc)
+    med = statistics.median
+    draft_gbs = dbytes / (med(t_draft) * 1e-3) / 1e9
+    verify_gbs = vbytes / (med(t_ver) * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers: copy this round's
+    # inputs from pinned host memory, run the round, read the result back
+    e2e = None
+    if not args.no_e2e:
+        host = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
+                for k in ("base", "target", "anchor", "u_draft", "u_accept", "u_resample", "conf")}
+        out_host = torch.empty(B * (K + 1) + B, dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * 4
+        e2e_steps = max(2, min(args.steps, 10))
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(e2e_steps):
+                for k2, t in host.items():
+                    dst = d[k2].view(-1) if k2 != "target" else d[k2].view(-1)
+                    dst.copy_(t.view(-1), non_blocking=True)
+                rnd.run_round(d, bufs, stream)
+                out_host[: B * (K + 1)].copy_(bufs.out_tokens.view(-1), non_blocking=True)
+                out_host[B * (K + 1):].copy_(bufs.n_out.view(-1), non_blocking=True)
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = ev0.elapsed_time(ev1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": e2e_steps * world / (e2e_ms / 1000.0), "unit": "rounds/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "note": "Markov factors are model weights kept resident; per-round logits, confidences "
+                       "and uniforms are copied in, emitted tokens copied out"}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(inp, seconds=args.cpu_seconds)
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            tj = json.load(f)
+        if tj.get("workload") == w.name and tj.get("kernel_version") == "draft-generic-v1":
+            traffic = tj.get("draft_bytes_per_launch")
+    line = {
+        "metric": "draft+schedule+verify rounds/sec", "value": value, "unit": "rounds/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32",
+        "dtype_detail": "fp32 logits, bf16 Markov factors with fp32 accumulation, fp64 vocabulary sums",
+        "data": "synthetic", "config": config_of(w),
+        "tokens_per_s": value * float(n_out.sum()),
+        "stages_ms_median": {"draft": med(t_draft), "schedule": med(t_sched), "verify": med(t_ver)},
+        "round_ms": {"median": med(t_round), "p10": float(np.percentile(t_round, 10)),
+                     "p90": float(np.percentile(t_round, 90))},
+        "roofline": {"bound": "hbm", "kernel": "dspark_markov_draft", "achieved": draft_gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": draft_gbs / peaks["hbm_gbs"],
+                     "traffic": traffic, "algorithmic_bytes": dbytes, "peak_source": peaks["source"]},
+        "roofline_verify": {"bound": "hbm", "achieved": verify_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": verify_gbs / peaks["hbm_gbs"], "algorithmic_bytes": vbytes},
+        "round_stats": {"verify_tokens": int((L + 1).sum()), "accepted_mean": float(acc.mean()),
+                        "emitted_per_round": int(n_out.sum())},
+        "gpu_launches": launches_per_round * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cb,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen3")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,149 @@
+/*
+ * dspark.h -- C ABI of the per-round hot path of DSpark-style speculative
+ * decoding on one B200 (sm_100a): semi-autoregressive Markov draft,
+ * confidence-scheduled verify lengths, lossless rejection-sampling verify.
+ *
+ * Sources (four web pages on DeepSeek's DSpark; titles abbreviated):
+ *   [Thread] sina.cn, "Fireworks AI CTO Dzhulgakov explains DSpark", items 1-10
+ *   [QbitAI] hzrcw.cc, "DSpark: ten concepts are enough", headed sections
+ *   [Essay]  10100.com, "speculative decoding is not making the model think less"
+ *   [Tags]   wangjunjian.com, tag page "speculative-decoding"
+ *
+ * Conventions (all entry points):
+ *   - Every array pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned, row-major, densely packed. The library allocates nothing and
+ *     keeps no state between calls apart from what lives in `workspace`.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.
+ *   - Argument errors (NULL pointer, size out of range, misalignment,
+ *     workspace too small) return DSPARK_ERR_INVALID_ARG before anything is
+ *     launched. Launch failures return DSPARK_ERR_CUDA.
+ *   - Errors found on the device (a token id outside [0,V), a verify length
+ *     outside [0,K], a device-wide wait that ran out of time) are recorded in
+ *     the workspace's error word; read them with dspark_read_device_error.
+ *     Kernels that hit such an error stop early and leave outputs undefined.
+ *   - One workspace per stream: calls that share a workspace must be ordered
+ *     on one stream. Zero a new workspace once with dspark_workspace_init.
+ *   - Limits: 1 <= B <= 65536, 1 <= K <= 32, 8 <= V <= 2^24 with V % 8 == 0,
+ *     1 <= r <= 512, B*K <= 16384 for dspark_schedule.
+ */
+#ifndef DSPARK_H_
+#define DSPARK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dspark_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  DSPARK_OK = 0,
+  DSPARK_ERR_INVALID_ARG = 1,
+  DSPARK_ERR_UNSUPPORTED = 2,
+  DSPARK_ERR_CUDA = 3,
+  DSPARK_ERR_TIMEOUT = 4,       /* a device-wide wait gave up (device error word) */
+  DSPARK_ERR_DEVICE_ASSERT = 5  /* an index check failed on the device (device error word) */
+} dspark_status;
+
+typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype;
+
+/* Bytes of workspace that dspark_markov_draft, dspark_schedule and
+ * dspark_verify need for these sizes (the maximum of the three, so one
+ * workspace serves a whole round). Returns 0 if the sizes are out of range. */
+size_t dspark_workspace_bytes(int B, int K, int V, int r);
+
+/* Zero `ws_bytes` bytes of a fresh workspace on `stream` (clears the error word). */
+dspark_status dspark_workspace_init(void* workspace, size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * Semi-autoregressive draft with the low-rank Markov head.
+ * [QbitAI] sections "DSpark = Eagle + DFlash" and "a cheaper sequential
+ * module: the Markov head"; [Essay] section "parallel drafts are fast ...";
+ * [Tags] DSpark summary, "semi-autoregressive generation".
+ *
+ * For i = 1..K in order, for every request b:
+ *   z[b,i,:]  = base_logits[b,i,:] + A[t_{b,i-1},:] . Bf        (t_{b,0} = anchor[b])
+ *   q         = softmax(z[b,i,:])
+ *   t_{b,i}   = smallest v with sum_{v'<=v} q_{v'} > u_draft[b,i]*sum(q)
+ *   q_tok     = q(t_{b,i}),  lse_q = log sum exp z[b,i,:]
+ *
+ * base_logits [B,K,V] f32; A [V,r] and Bf [r,V] of factor_dtype (bf16 is
+ * IEEE bfloat16 bits); anchor [B] i32 in [0,V); u_draft [B,K] f32 in [0,1).
+ * Outputs: draft_tokens [B,K] i32; q_tok [B,K] f32; lse_q [B,K] f64 (the
+ * normaliser is kept in fp64 because verification forms max(0, p - q), which a
+ * common fp32 rounding of the normaliser would shift); z [B,K,V] f32.
+ * Sums over the vocabulary are taken in fp64 of fp32 exponentials.
+ */
+dspark_status dspark_markov_draft(const float* base_logits, const void* A, const void* Bf,
+                                  dspark_dtype factor_dtype, int r, const int32_t* anchor,
+                                  const float* u_draft, int B, int K, int V,
+                                  int32_t* draft_tokens, float* q_tok, double* lse_q, float* z,
+                                  void* workspace, size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * Confidence-scheduled verify lengths.
+ * [QbitAI] section "variable-length drafts and hardware-aware scheduling"
+ * (a confidence head scores each position's survival; a pre-measured
+ * throughput curve picks each request's verify length, all on the GPU) and
+ * section "online drafter calibration" (sequential temperature scaling);
+ * [Thread] items 4 and 9 (time per token; load-dependent draft length).
+ *
+ *   s[b,j] = 1/(1+exp(-conf_logits[b,j]/temps[j])),  P[b,j] = prod_{k<=j} s[b,k]
+ *   Rank items (b,j) by P descending, then j ascending, then b ascending; S_m =
+ *   sum of the first m; choose the smallest m* maximising (B + S_m)/T(B+m) over
+ *   0 <= m <= min(B*K, n_prof-B), where T(n) = profile_ms[n-1];
+ *   verify_len[b] = number of request b's items among the first m*.
+ *
+ * conf_logits [B,K] f32; temps [K] f32 > 0; profile_ms [n_prof] f32 (n_prof >= B).
+ * Outputs: verify_len [B] i32 in [0,K]; survival [B,K] f32 (P);
+ * row_start [B] i64 (exclusive scan of verify_len+1: packed target-row
+ * offsets); n_tokens [1] i32 (sum of verify_len+1).
+ */
+dspark_status dspark_schedule(const float* conf_logits, const float* temps, const float* profile_ms,
+                              int n_prof, int B, int K, int32_t* verify_len, float* survival,
+                              int64_t* row_start, int32_t* n_tokens, void* workspace,
+                              size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * Lossless rejection-sampling verification.
+ * [QbitAI] section "speculative decoding" (check candidates one by one,
+ * keep the longest accepted prefix, resample at the first divergence, output
+ * distributed exactly as the target); [Tags] "Speculative Decoding" steps
+ * 3-5 (compare probabilities with a random number; sample from the target if
+ * all pass, else from an adjusted distribution).
+ *
+ * Request b's target rows are target_logits[row_start[b] + rho], rho = 0..L_b
+ * (L_b = verify_len[b]); p_j = softmax(row j-1). Draft j <= L_b is accepted iff
+ * u_accept[b,j]*q_tok[b,j] < p_j(t_j); j* = first rejection. If j* exists the
+ * final token is drawn with u_resample[b] from max(0, p_j* - q_j*) renormalised
+ * (q_j* = exp(z[b,j*] - lse_q[b,j*])), else from p_{L_b+1} (row L_b, bonus).
+ *
+ * target_logits [*,V] f32 (dense [B,K+1,V] is row_start[b] = b*(K+1));
+ * z, lse_q, q_tok, draft_tokens as produced by dspark_markov_draft;
+ * verify_len [B] i32; u_accept [B,K] and u_resample [B] f32 in [0,1).
+ * Outputs: accepted [B] i32 (accepted drafts); out_tokens [B,K+1] i32
+ * (accepted drafts, then the final token, then -1); n_out [B] i32 (accepted+1).
+ */
+dspark_status dspark_verify(const float* target_logits, const int64_t* row_start, const float* z,
+                            const double* lse_q, const float* q_tok, const int32_t* draft_tokens,
+                            const int32_t* verify_len, const float* u_accept,
+                            const float* u_resample, int B, int K, int V, int32_t* accepted,
+                            int32_t* out_tokens, int32_t* n_out, void* workspace, size_t ws_bytes,
+                            dspark_stream_t stream);
+
+/* Synchronise `stream`, return the status recorded in the workspace's error
+ * word (DSPARK_OK if none) and clear it; *detail (if non-NULL) receives the
+ * offending value or the index of the wait that timed out. */
+dspark_status dspark_read_device_error(void* workspace, dspark_stream_t stream, uint32_t* detail);
+
+/* Static, human-readable name of a status. */
+const char* dspark_status_string(dspark_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H_ */

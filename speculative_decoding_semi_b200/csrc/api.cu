@@ -1,0 +1,178 @@
+// C ABI of libdspark: argument validation, workspace layout and launches.
+// Every entry point checks its arguments before launching anything, enqueues
+// work on the caller's stream and returns without synchronising.
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dspark {
+cudaError_t launch_draft_generic(DraftArgs a, int G, cudaStream_t stream);
+int draft_grid_size(int V, int sms);
+}  // namespace dspark
+
+using namespace dspark;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool sizes_ok(int B, int K, int V) {
+  return B >= 1 && B <= kMaxB && K >= 1 && K <= kMaxK && V >= 8 && V <= kMaxV && (V % 8) == 0;
+}
+
+size_t scratch_bytes(int B, int K, int V, int r) {
+  return std::max({draft_scratch_bytes(B, K, V, r), verify_scratch_bytes(B, K, V),
+                   schedule_scratch_bytes(B, K)});
+}
+
+dspark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t dspark_workspace_bytes(int B, int K, int V, int r) {
+  if (!sizes_ok(B, K, V) || r < 1 || r > kMaxR) return 0;
+  return kScratchOffset + align_up(scratch_bytes(B, K, V, r), 256);
+}
+
+dspark_status dspark_workspace_init(void* workspace, size_t ws_bytes, dspark_stream_t stream) {
+  if (workspace == nullptr || ws_bytes < kScratchOffset || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(workspace, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_markov_draft(const float* base_logits, const void* A, const void* Bf,
+                                  dspark_dtype factor_dtype, int r, const int32_t* anchor,
+                                  const float* u_draft, int B, int K, int V, int32_t* draft_tokens,
+                                  float* q_tok, double* lse_q, float* z, void* workspace,
+                                  size_t ws_bytes, dspark_stream_t stream) {
+  if (!sizes_ok(B, K, V) || r < 1 || r > kMaxR) return DSPARK_ERR_INVALID_ARG;
+  if (factor_dtype != DSPARK_F32 && factor_dtype != DSPARK_BF16) return DSPARK_ERR_INVALID_ARG;
+  const void* ptrs[] = {base_logits, A, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, z, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < dspark_workspace_bytes(B, K, V, r)) return DSPARK_ERR_INVALID_ARG;
+  if (2u * K * sizeof(unsigned) > kSyncBytes) return DSPARK_ERR_INVALID_ARG;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DSPARK_ERR_CUDA;
+  const int G = draft_grid_size(V, sms);
+
+  DraftArgs a{};
+  a.base = base_logits;
+  a.A = A;
+  a.Bf = Bf;
+  a.bf16 = factor_dtype == DSPARK_BF16;
+  a.r = r;
+  a.anchor = anchor;
+  a.u = u_draft;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.tokens = draft_tokens;
+  a.q_tok = q_tok;
+  a.lse_q = lse_q;
+  a.z = z;
+  a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
+  a.sync = reinterpret_cast<unsigned*>(ws + kSyncOffset);
+  char* scratch = ws + kScratchOffset;
+  a.part_m = reinterpret_cast<float*>(scratch);
+  a.part_S = reinterpret_cast<double*>(scratch + align_up(static_cast<size_t>(B) * G * sizeof(float), 256));
+
+  cudaError_t e = cudaMemsetAsync(a.sync, 0, 2u * K * sizeof(unsigned), s);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  return from_cuda(launch_draft_generic(a, G, s));
+}
+
+dspark_status dspark_schedule(const float* conf_logits, const float* temps, const float* profile_ms,
+                              int n_prof, int B, int K, int32_t* verify_len, float* survival,
+                              int64_t* row_start, int32_t* n_tokens, void* workspace, size_t ws_bytes,
+                              dspark_stream_t stream) {
+  if (B < 1 || B > kMaxB || K < 1 || K > kMaxK || static_cast<long long>(B) * K > kMaxScheduleItems)
+    return DSPARK_ERR_INVALID_ARG;
+  if (n_prof < B) return DSPARK_ERR_INVALID_ARG;
+  const void* ptrs[] = {conf_logits, temps, profile_ms, verify_len, survival, row_start, n_tokens, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < kScratchOffset + schedule_scratch_bytes(B, K)) return DSPARK_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  ScheduleArgs a{};
+  a.conf = conf_logits;
+  a.temps = temps;
+  a.profile = profile_ms;
+  a.n_prof = n_prof;
+  a.B = B;
+  a.K = K;
+  a.verify_len = verify_len;
+  a.survival = survival;
+  a.row_start = row_start;
+  a.n_tokens = n_tokens;
+  a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
+  return from_cuda(launch_schedule(a, ws + kScratchOffset, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_verify(const float* target_logits, const int64_t* row_start, const float* z,
+                            const double* lse_q, const float* q_tok, const int32_t* draft_tokens,
+                            const int32_t* verify_len, const float* u_accept, const float* u_resample,
+                            int B, int K, int V, int32_t* accepted, int32_t* out_tokens, int32_t* n_out,
+                            void* workspace, size_t ws_bytes, dspark_stream_t stream) {
+  if (!sizes_ok(B, K, V)) return DSPARK_ERR_INVALID_ARG;
+  const void* ptrs[] = {target_logits, row_start, z, lse_q, q_tok, draft_tokens, verify_len,
+                        u_accept, u_resample, accepted, out_tokens, n_out, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < kScratchOffset + verify_scratch_bytes(B, K, V)) return DSPARK_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  VerifyArgs a{};
+  a.target = target_logits;
+  a.row_start = row_start;
+  a.z = z;
+  a.lse_q = lse_q;
+  a.q_tok = q_tok;
+  a.tokens = draft_tokens;
+  a.verify_len = verify_len;
+  a.u_accept = u_accept;
+  a.u_resample = u_resample;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.accepted = accepted;
+  a.out_tokens = out_tokens;
+  a.n_out = n_out;
+  a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
+  return from_cuda(launch_verify(a, ws + kScratchOffset, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_read_device_error(void* workspace, dspark_stream_t stream, uint32_t* detail) {
+  if (workspace == nullptr || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned host[2] = {0, 0};
+  if (cudaMemcpyAsync(host, workspace, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (detail) *detail = host[1];
+  if (host[0] != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(host), s) != cudaSuccess) return DSPARK_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  return static_cast<dspark_status>(host[0]);
+}
+
+const char* dspark_status_string(dspark_status status) {
+  switch (status) {
+    case DSPARK_OK: return "ok";
+    case DSPARK_ERR_INVALID_ARG: return "invalid argument";
+    case DSPARK_ERR_UNSUPPORTED: return "unsupported";
+    case DSPARK_ERR_CUDA: return "CUDA error";
+    case DSPARK_ERR_TIMEOUT: return "device-wide wait timed out";
+    case DSPARK_ERR_DEVICE_ASSERT: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

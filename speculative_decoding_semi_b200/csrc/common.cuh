@@ -1,0 +1,215 @@
+// Device helpers shared by the draft, schedule and verify kernels:
+// the workspace error word, bounded device-wide waits, block reductions and
+// scans in fp32/fp64, and the workspace layout.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+// ---------------------------------------------------------------- limits
+constexpr int kMaxB = 65536;
+constexpr int kMaxK = 32;
+constexpr int kMaxV = 1 << 24;
+constexpr int kMaxR = 512;
+constexpr int kMaxScheduleItems = 16384;
+constexpr int kMaxGrid = 256;        // CTAs of the persistent draft kernel (>= SM count)
+constexpr int kVerifySeg = 4096;     // vocabulary segment of the verify kernels
+
+// -------------------------------------------------------- workspace layout
+// [0, 256)      error word: u32 code, u32 detail
+// [256, 4352)   counters of the device-wide waits (cleared by every draft launch)
+// [4352, ...)   per-call scratch (draft partials / verify partials / schedule
+//               arrays); calls on one stream reuse it in turn.
+constexpr size_t kErrOffset = 0;
+constexpr size_t kSyncOffset = 256;
+constexpr size_t kSyncBytes = 4096;
+constexpr size_t kScratchOffset = kSyncOffset + kSyncBytes;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------ error word
+constexpr unsigned kWaitIterLimit = 1u << 26;           // spins before a wait gives up
+constexpr unsigned long long kWaitBudgetNs = 1000000000ull;  // 1 s of device time
+
+__device__ __forceinline__ void set_error(unsigned* err, unsigned code, unsigned detail) {
+  if (atomicCAS(err, 0u, code) == 0u) atomicExch(err + 1, detail);
+}
+
+__device__ __forceinline__ unsigned error_code(const unsigned* err) {
+  return *reinterpret_cast<const volatile unsigned*>(err);
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Spin (one thread) until *ctr >= target. Gives up when the error word is set
+// by anyone, after kWaitIterLimit polls, or after kWaitBudgetNs; in the last
+// two cases it records DSPARK_ERR_TIMEOUT with `where`. Returns true on success.
+static __device__ __noinline__ bool wait_at_least(const unsigned* ctr, unsigned target, unsigned* err,
+                                           unsigned where) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (unsigned it = 0; it < kWaitIterLimit; ++it) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if ((it & 31u) == 31u) {
+      if (error_code(err) != 0u) return false;
+      if (globaltimer_ns() - t0 > kWaitBudgetNs) break;
+    }
+    __nanosleep(40);
+  }
+  set_error(err, DSPARK_ERR_TIMEOUT, where);
+  return false;
+}
+
+// CTA-wide: thread 0 waits, the result is broadcast; all threads then see the
+// producers' writes (acquire by thread 0, ordered for the CTA by the barrier).
+__device__ __forceinline__ bool cta_wait_at_least(const unsigned* ctr, unsigned target, unsigned* err,
+                                                  unsigned where, int* s_flag) {
+  if (threadIdx.x == 0) {
+    bool ok = wait_at_least(ctr, target, err, where);
+    __threadfence();
+    *s_flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  bool ok = *s_flag != 0;
+  __syncthreads();
+  return ok;
+}
+
+// CTA-wide release: every thread's prior global writes become visible before
+// the counter moves.
+__device__ __forceinline__ void cta_release_add(unsigned* ctr, unsigned v) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_gpu_add(ctr, v);
+  }
+}
+
+// ----------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_min_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_max_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide reductions; `red` is shared scratch of >= 32 elements. All
+// threads of the block must call; every thread gets the result.
+template <int NT>
+__device__ __forceinline__ float block_max(float v, float* red) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < NT / 32) ? red[l] : -INFINITY;
+  v = warp_max(v);
+  return v;
+}
+template <int NT>
+__device__ __forceinline__ double block_sum(double v, double* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < NT / 32) ? red[l] : 0.0;
+  v = warp_sum(v);
+  return v;
+}
+template <int NT>
+__device__ __forceinline__ int block_min_int(int v, int* red) {
+  v = warp_min_int(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < NT / 32) ? red[l] : 0x7fffffff;
+  v = warp_min_int(v);
+  return v;
+}
+template <int NT>
+__device__ __forceinline__ int block_max_int(int v, int* red) {
+  v = warp_max_int(v);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < NT / 32) ? red[l] : -0x7fffffff;
+  v = warp_max_int(v);
+  return v;
+}
+
+// Inclusive scan of fp64 within a warp.
+__device__ __forceinline__ double warp_inclusive_scan(double v) {
+  const int l = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    double n = __shfl_up_sync(0xffffffffu, v, o);
+    if (l >= o) v += n;
+  }
+  return v;
+}
+
+// Block-wide exclusive scan of fp64 (thread order); returns the exclusive
+// prefix, writes the block total to *total. `red` >= 33 doubles of shared.
+template <int NT>
+__device__ __forceinline__ double block_exclusive_scan(double v, double* red, double* total) {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  double inc = warp_inclusive_scan(v);
+  double exw = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (l == 0) exw = 0.0;
+  __syncthreads();
+  if (l == 31) red[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    double s = (l < NT / 32) ? red[l] : 0.0;
+    double si = warp_inclusive_scan(s);
+    double se = __shfl_up_sync(0xffffffffu, si, 1);
+    if (l == 0) se = 0.0;
+    if (l < NT / 32) red[l] = se;
+    if (l == NT / 32 - 1) red[32] = si;
+  }
+  __syncthreads();
+  double ex = red[w] + exw;
+  *total = red[32];
+  __syncthreads();
+  return ex;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<unsigned>(b) << 16);
+}
+
+}  // namespace dspark

@@ -1,0 +1,82 @@
+// Launchers of the draft, schedule and verify kernels (internal to libdspark).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+struct DraftArgs {
+  const float* base;
+  const void* A;
+  const void* Bf;
+  int bf16;
+  int r;
+  const int32_t* anchor;
+  const float* u;
+  int B, K, V;
+  int32_t* tokens;
+  float* q_tok;
+  double* lse_q;
+  float* z;
+  unsigned* err;
+  unsigned* sync;   // 2*K counters
+  float* part_m;    // [B][G]
+  double* part_S;   // [B][G]
+};
+
+struct VerifyDecision {
+  int acc;    // accepted drafts
+  int mode;   // 0 = residual at row acc, 1 = bonus at row acc (= L_b)
+  double M;   // max logit of the final row
+  double W;   // sum exp(x - M) of the final row
+};
+
+struct VerifyArgs {
+  const float* target;
+  const int64_t* row_start;
+  const float* z;
+  const double* lse_q;
+  const float* q_tok;
+  const int32_t* tokens;
+  const int32_t* verify_len;
+  const float* u_accept;
+  const float* u_resample;
+  int B, K, V, nseg;
+  int32_t* accepted;
+  int32_t* out_tokens;
+  int32_t* n_out;
+  unsigned* err;
+  float* rp_m;          // [B*(K+1)][nseg]
+  double* rp_S;         // [B*(K+1)][nseg]
+  float* x_tok;         // [B*K]
+  double* seg_w;        // [B][nseg]
+  VerifyDecision* dec;  // [B]
+};
+
+struct ScheduleArgs {
+  const float* conf;
+  const float* temps;
+  const float* profile;
+  int n_prof, B, K;
+  int32_t* verify_len;
+  float* survival;
+  int64_t* row_start;
+  int32_t* n_tokens;
+  unsigned* err;
+  int32_t* rank;        // [B*K]
+  double* sorted_P;     // [B*K]
+};
+
+size_t draft_scratch_bytes(int B, int K, int V, int r);
+size_t verify_scratch_bytes(int B, int K, int V);
+size_t schedule_scratch_bytes(int B, int K);
+
+cudaError_t launch_draft(DraftArgs a, char* scratch, cudaStream_t stream);
+cudaError_t launch_verify(VerifyArgs a, char* scratch, cudaStream_t stream);
+cudaError_t launch_schedule(ScheduleArgs a, char* scratch, cudaStream_t stream);
+
+}  // namespace dspark

@@ -56,6 +56,8 @@ WORKLOADS = (
 
 
 def workload(key) -> Workload:
+    if isinstance(key, Workload):
+        return key
     if isinstance(key, int):
         return WORKLOADS[key]
     for w in WORKLOADS:
@@ -123,6 +125,12 @@ def _conf(w: Workload, rng, sigma) -> np.ndarray:
     else:
         mean = np.ones((w.B, 1), np.float32)
     return (mean + rng.standard_normal(size=(w.B, w.K), dtype=np.float32)).astype(np.float32)
+
+
+def custom(like, **sizes) -> Workload:
+    """A workload with another workload's recipe (sigma, confidence, profile
+    shape, factor dtype) and the given sizes, e.g. custom(1, B=8, V=37000)."""
+    return dataclasses.replace(workload(like), **sizes)
 
 
 def make_round(key, seed: int | None = None, with_target: bool = True) -> dict:

@@ -1,0 +1,192 @@
+"""GPU-vs-oracle comparison of one round (test infrastructure).
+
+Integer outputs must match exactly, except where the oracle's own decision
+margin is below MARGIN (1e-5): inverse-CDF margin d < 1e-5, accept margin
+|u - p/q| < 1e-5, or a scheduler near-tie (|P_(m*) - P_(m*+1)| < 1e-5 P_(m*)
+or a runner-up objective within 1e-5). Such mismatches are counted as
+excused and their pooled rate must stay under 0.1% of decisions; any other
+mismatch fails. After an excused mismatch the oracle continues from the GPU's
+choice (teacher forcing), so one near-tie counts once.
+Float outputs: q_tok and survival within 2e-3 relative, lse_q within 2e-3
+absolute; z within 1e-4 absolute + 1e-5 relative (fp32 rounding of base +
+bias, with the bias accumulated in fp32).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+
+MARGIN = 1e-5
+RATE = 1e-3
+
+
+@dataclasses.dataclass
+class Tally:
+    decisions: int = 0
+    excused: int = 0
+    flagged: int = 0
+    failures: list = dataclasses.field(default_factory=list)
+
+    def add(self, other: "Tally"):
+        self.decisions += other.decisions
+        self.excused += other.excused
+        self.flagged += other.flagged
+        self.failures += other.failures
+
+    def check(self, min_rate_decisions: int = 2000):
+        assert not self.failures, self.failures[:10]
+        limit = max(1, int(RATE * self.decisions)) if self.decisions < min_rate_decisions else RATE * self.decisions
+        assert self.excused <= limit, (self.excused, self.decisions)
+
+
+def compare_draft(inp, gpu, requests, tally: Tally, check_z=True):
+    """gpu: dict of numpy outputs for the sampled `requests` (tokens, q_tok, lse_q, z)."""
+    base = inp["base"][requests]
+    d = oracle.draft(base, inp["A"], inp["Bf"], inp["anchor"][requests], inp["u_draft"][requests],
+                     teacher=gpu["tokens"].astype(np.int64), keep_z=True)
+    mism = d["t"] != gpu["tokens"]
+    small = d["margin"] < MARGIN
+    tally.decisions += mism.size
+    tally.flagged += int(small.sum())
+    tally.excused += int((mism & small).sum())
+    bad = np.argwhere(mism & ~small)
+    for b, i in bad[:5]:
+        tally.failures.append(("draft token", int(requests[b]), int(i), int(d["t"][b, i]), int(gpu["tokens"][b, i]),
+                               float(d["margin"][b, i])))
+    rel = np.abs(gpu["q_tok"] - d["q_tok"]) / np.maximum(d["q_tok"], 1e-300)
+    if rel.max() > 2e-3:
+        tally.failures.append(("q_tok rel", float(rel.max())))
+    err = np.abs(gpu["lse_q"] - d["lse"]).max()
+    if err > 2e-3:
+        tally.failures.append(("lse_q abs", float(err)))
+    if check_z:
+        zerr = np.abs(gpu["z"].astype(np.float64) - d["z"]) - 1e-5 * np.abs(d["z"])
+        if zerr.max() > 1e-4:
+            idx = np.unravel_index(np.argmax(zerr), zerr.shape)
+            tally.failures.append(("z", float(zerr.max()), idx))
+    return d
+
+
+def compare_schedule(inp, gpu, tally: Tally):
+    P = oracle.survival(inp["conf"], inp["temps"])
+    s = oracle.schedule(P, inp["profile"])
+    rel = np.abs(gpu["survival"] - P) / P
+    if rel.max() > 2e-3:
+        tally.failures.append(("survival rel", float(rel.max())))
+    B = P.shape[0]
+    tally.decisions += B
+    L = gpu["verify_len"]
+    if not np.array_equal(L, s["verify_len"]):
+        if s["gap_item"] < MARGIN or s["gap_obj"] < MARGIN:
+            tally.excused += int((L != s["verify_len"]).sum())
+        else:
+            tally.failures.append(("verify_len", np.argwhere(L != s["verify_len"]).ravel()[:5].tolist(),
+                                   float(s["gap_item"]), float(s["gap_obj"])))
+    # the GPU's own offsets must be the exclusive scan of its own lengths
+    exp_rs = np.concatenate([[0], np.cumsum(L.astype(np.int64) + 1)[:-1]])
+    if not np.array_equal(gpu["row_start"], exp_rs):
+        tally.failures.append(("row_start", gpu["row_start"][:5].tolist(), exp_rs[:5].tolist()))
+    if int(gpu["n_tokens"]) != int((L + 1).sum()):
+        tally.failures.append(("n_tokens", int(gpu["n_tokens"]), int((L + 1).sum())))
+    return s
+
+
+def compare_verify(inp, draft_oracle, gpu_draft, gpu, verify_len, requests, tally: Tally):
+    """Teacher-forced: the oracle verifies the GPU's tokens with the GPU's lengths."""
+    B, K, V = inp["base"].shape
+    rows = inp["target"].reshape(B * (K + 1), V)
+    rs = np.arange(B, dtype=np.int64) * (K + 1)
+    vo = oracle.verify(rows, rs, draft_oracle["z"], draft_oracle["lse"], draft_oracle["q_tok"],
+                       gpu_draft["tokens"], verify_len, inp["u_accept"], inp["u_resample"],
+                       requests=requests)
+    acc_g = gpu["accepted"]
+    vo2 = None
+    for idx, b in enumerate(requests):
+        Lb = int(verify_len[b])
+        margins = vo["accept_margin"][idx]
+        tally.decisions += len(margins)
+        tally.flagged += int(sum(m < MARGIN for m in margins))
+        ao, ag = int(vo["accepted"][idx]), int(acc_g[idx])
+        if ao != ag:
+            j = min(ao, ag)  # first position where the decisions differ (0-based)
+            if j < len(margins) and margins[j] < MARGIN:
+                tally.excused += 1
+            else:
+                tally.failures.append(("accepted", int(b), ao, ag, margins[j] if j < len(margins) else None))
+        if not (1 <= gpu["n_out"][idx] <= Lb + 1) or gpu["n_out"][idx] != ag + 1:
+            tally.failures.append(("n_out", int(b), int(gpu["n_out"][idx]), ag))
+        if not np.array_equal(gpu["out_tokens"][idx, :ag], gpu_draft["tokens"][idx, :ag]):
+            tally.failures.append(("prefix", int(b)))
+        if np.any(gpu["out_tokens"][idx, ag + 1:] != -1):
+            tally.failures.append(("padding", int(b)))
+    # final token, teacher-forced on the GPU's acceptance count
+    vo2 = oracle.verify(rows, rs, draft_oracle["z"], draft_oracle["lse"], draft_oracle["q_tok"],
+                        gpu_draft["tokens"], verify_len, inp["u_accept"], inp["u_resample"],
+                        forced_accepted=_full(acc_g, requests, B), requests=requests)
+    for idx, b in enumerate(requests):
+        tally.decisions += 1
+        m = vo2["final_margin"][idx]
+        tally.flagged += int(m < MARGIN)
+        fg = int(gpu["out_tokens"][idx, acc_g[idx]])
+        if fg != int(vo2["final"][idx]):
+            if m < MARGIN:
+                tally.excused += 1
+            else:
+                tally.failures.append(("final", int(b), int(vo2["final"][idx]), fg, float(m), vo2["final_mode"][idx]))
+    return vo2
+
+
+def _full(vals, requests, B):
+    out = np.zeros(B, np.int64)
+    out[np.asarray(requests)] = vals
+    return out
+
+
+def gpu_round(inp, requests=None, packed=False):
+    """Run draft -> schedule -> verify through the library; numpy outputs."""
+    from speculative_decoding_semi_b200 import round as rnd
+
+    B, K, V = inp["base"].shape
+    r = inp["A"].shape[1]
+    d = rnd.to_device(inp)
+    bufs = rnd.RoundBuffers(B, K, V, r)
+    rnd.draft(d, bufs)
+    rnd.schedule(d, bufs)
+    if packed:
+        L = bufs.verify_len.cpu().numpy()
+        rs = bufs.row_start.cpu().numpy()
+        tgt = torch.from_numpy(synth.pack_rows(inp["target"], L, rs)).cuda()
+        rnd.verify(d, bufs, target=tgt, row_start=bufs.row_start)
+    else:
+        rnd.verify(d, bufs)
+    torch.cuda.synchronize()
+    from speculative_decoding_semi_b200 import dspark_read_device_error
+    st, detail = dspark_read_device_error(bufs.workspace)
+    assert st == 0, (st, hex(detail))
+    reqs = np.arange(B) if requests is None else np.asarray(requests)
+    ridx = torch.as_tensor(reqs, device=bufs.z.device)
+    take = lambda t: t.index_select(0, ridx).cpu().numpy()
+    out = {
+        "draft": {"tokens": take(bufs.draft_tokens), "q_tok": take(bufs.q_tok), "lse_q": take(bufs.lse_q),
+                  "z": take(bufs.z) if len(reqs) * K * V <= 64 * 8 * 151936 else None},
+        "schedule": {"verify_len": bufs.verify_len.cpu().numpy(), "survival": bufs.survival.cpu().numpy(),
+                     "row_start": bufs.row_start.cpu().numpy(), "n_tokens": bufs.n_tokens.cpu().numpy()[0]},
+        "verify": {"accepted": take(bufs.accepted), "out_tokens": take(bufs.out_tokens), "n_out": take(bufs.n_out)},
+    }
+    return out
+
+
+def check_round(inp, requests=None, packed=False, tally: Tally | None = None, check_z=True):
+    B = inp["base"].shape[0]
+    reqs = np.arange(B) if requests is None else np.asarray(requests)
+    g = gpu_round(inp, reqs, packed=packed)
+    t = Tally() if tally is None else tally
+    d = compare_draft(inp, g["draft"], reqs, t, check_z=check_z and g["draft"]["z"] is not None)
+    compare_schedule(inp, g["schedule"], t)
+    compare_verify(inp, d, g["draft"], g["verify"], g["schedule"]["verify_len"], reqs, t)
+    return t, g

@@ -1,0 +1,123 @@
+"""GPU path (through the C ABI) against the CPU oracle, element by element.
+
+Sizes: the tiny workload over many seeds; medium sizes that span many
+vocabulary chunks and verify segments with ragged tails (V not a multiple of
+the 4096-wide segment); every full-size workload (all requests where the
+oracle is quick, a sample of requests otherwise); the exhaustive V=8
+enumeration; and edge cases (B=1, K=1, V=8, every verify length 0, packed
+ragged target rows, invalid indices reported through the error word).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import enumeration as en
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_many_seeds():
+    t = parity.Tally()
+    for seed in range(40):
+        inp = synth.make_round(0, seed=5000 + seed)
+        parity.check_round(inp, tally=t)
+    t.check()
+
+
+@pytest.mark.parametrize("like,sizes", [
+    (1, dict(B=12, K=5, V=37000, r=64, n_prof=256)),
+    (0, dict(B=9, K=6, V=20488, r=32, n_prof=128)),
+    (1, dict(B=3, K=16, V=4104, r=256, n_prof=64)),
+    (1, dict(B=130, K=2, V=8200, r=16, n_prof=512)),
+])
+def test_medium_ragged(like, sizes):
+    t = parity.Tally()
+    w = synth.custom(like, **sizes)
+    for seed in range(3):
+        parity.check_round(synth.make_round(w, seed=77 + seed), tally=t)
+    t.check()
+
+
+def test_packed_target_rows():
+    w = synth.custom(1, B=16, K=6, V=12344, r=32, n_prof=80)
+    t = parity.Tally()
+    for seed in range(2):
+        parity.check_round(synth.make_round(w, seed=900 + seed), packed=True, tally=t)
+    t.check()
+
+
+def test_edge_single_request_single_position():
+    for like, V in ((0, 8), (1, 64), (1, 151936)):
+        w = synth.custom(like, B=1, K=1, V=V, r=8, n_prof=4)
+        t = parity.Tally()
+        for seed in range(3):
+            parity.check_round(synth.make_round(w, seed=seed), tally=t)
+        t.check()
+
+
+def test_edge_all_verify_lengths_zero():
+    w = synth.custom(1, B=10, K=4, V=4096, r=16, n_prof=40)
+    inp = synth.make_round(w, seed=3)
+    inp["profile"] = (1.0 + 1000.0 * np.maximum(np.arange(1, 41) - 10, 0)).astype(np.float32)
+    t, g = parity.check_round(inp)
+    t.check()
+    assert np.all(g["schedule"]["verify_len"] == 0)
+    assert np.all(g["verify"]["n_out"] == 1)
+
+
+def _gpu_enumeration(prob, L):
+    from speculative_decoding_semi_b200 import round as rnd
+    batch = en.build_batch(prob, L)
+    n = len(batch["weight"])
+    inp = {"base": batch["base"], "A": prob["A"], "Bf": prob["Bf"], "anchor": batch["anchor"],
+           "u_draft": batch["u_draft"], "u_accept": batch["u_accept"], "u_resample": batch["u_resample"],
+           "target": batch["target"]}
+    d = rnd.to_device(inp)
+    bufs = rnd.RoundBuffers(n, en.K, en.V, en.R)
+    rnd.draft(d, bufs)
+    vl = torch.full((n,), L, dtype=torch.int32, device="cuda")
+    rnd.verify(d, bufs, verify_len=vl)
+    torch.cuda.synchronize()
+    return batch, {k: getattr(bufs, k).cpu().numpy() for k in ("draft_tokens", "accepted", "out_tokens", "n_out")}
+
+
+@pytest.mark.parametrize("L", [0, 1, 2, 3])
+def test_exhaustive_v8_lossless_on_gpu(L):
+    prob = en.make_problem()
+    batch, g = _gpu_enumeration(prob, L)
+    assert np.array_equal(g["draft_tokens"], batch["path"])
+    joint = en.tally(batch, g["out_tokens"], g["n_out"])
+    en.check_lossless(prob, batch, joint, tol=1e-9)
+    en.check_accept_rate(prob, batch, g["accepted"], tol=1e-9)
+
+
+@pytest.mark.parametrize("key,sample", [("qwen3", None), ("latency", None), ("highconc", 8), ("mixed", 8)])
+def test_full_size_workloads(key, sample):
+    inp = synth.make_round(key)
+    B = inp["base"].shape[0]
+    reqs = None if sample is None else np.linspace(0, B - 1, sample).astype(int)
+    t, g = parity.check_round(inp, requests=reqs, check_z=sample is None)
+    t.check()
+
+
+def test_device_errors_reported():
+    from speculative_decoding_semi_b200 import dspark_read_device_error
+    from speculative_decoding_semi_b200 import round as rnd
+    w = synth.custom(1, B=4, K=3, V=1024, r=16, n_prof=32)
+    inp = synth.make_round(w, seed=1)
+    inp["anchor"] = inp["anchor"].copy()
+    inp["anchor"][2] = 5000  # outside [0, V)
+    d = rnd.to_device(inp)
+    bufs = rnd.RoundBuffers(4, 3, 1024, 16)
+    rnd.draft(d, bufs)
+    st, detail = dspark_read_device_error(bufs.workspace)
+    assert st == 5 and (detail & 0xFFFF) == 2
+    assert dspark_read_device_error(bufs.workspace)[0] == 0  # cleared
+    rnd.run_round(rnd.to_device(synth.make_round(w, seed=2)), bufs)
+    bad = torch.tensor([0, 1, 7, 2], dtype=torch.int32, device="cuda")  # 7 > K
+    rnd.verify(d, bufs, verify_len=bad)
+    st, detail = dspark_read_device_error(bufs.workspace)
+    assert st == 5 and (detail & 0xFFFF) == 2
