@@ -1,6 +1,6 @@
 """Build libdspark.so in-tree with nvcc for sm_100a (B200).
 
-Usage: python -m speculative_decoding_semi_b200.build [--verbose]
+Usage: python speculative_decoding_semi_b200/build.py [--verbose] [--ptxas]
 Each .cu under csrc/ is compiled in parallel to an object file under _build/,
 then linked into speculative_decoding_semi_b200/libdspark.so with the CUDA
 runtime linked statically (the library then needs only the driver at run time).
