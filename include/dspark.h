@@ -134,6 +134,30 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
                             int32_t* out_tokens, int32_t* n_out, void* workspace, size_t ws_bytes,
                             dspark_stream_t stream);
 
+/*
+ * dspark_schedule without a workspace, for callers that cannot allocate
+ * device memory (their allocator belongs to another framework, they run inside
+ * stream capture, or their hot path forbids cudaMalloc). The pages describe no
+ * such variant; it computes exactly what dspark_schedule computes, with the
+ * same kernels, and allocates nothing.
+ *
+ * Its scratch is one static device array of fixed size inside libdspark
+ * (room for DSPARK_STATIC_SCHEDULE_MAX_ITEMS items, about 192 KB), which every
+ * GPU that loads the library holds until the process exits. B*K above that
+ * limit returns DSPARK_ERR_INVALID_ARG; other argument rules are those of
+ * dspark_schedule. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current, so make the first
+ * call on each device before any stream capture. All calls share the one
+ * array, and each call fully rewrites what it reads back, so no state carries
+ * over between calls; calls that overlap on the GPU (two streams, or two
+ * threads) race on the array and must be serialised by the caller.
+ */
+#define DSPARK_STATIC_SCHEDULE_MAX_ITEMS 16384
+dspark_status dspark_schedule_static(const float* conf_logits, const float* temps,
+                                     const float* profile_ms, int n_prof, int B, int K,
+                                     int32_t* verify_len, float* survival, int64_t* row_start,
+                                     int32_t* n_tokens, dspark_stream_t stream);
+
 /* Synchronise `stream`, return the status recorded in the workspace's error
  * word (DSPARK_OK if none) and clear it; *detail (if non-NULL) receives the
  * offending value or the index of the wait that timed out. */

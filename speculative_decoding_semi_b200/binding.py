@@ -33,7 +33,7 @@ class DSparkError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m speculative_decoding_semi_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python speculative_decoding_semi_b200/build.py` "
             "(nvcc, sm_100a). There is no CPU fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, Z, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
@@ -49,6 +49,8 @@ def _load() -> ctypes.CDLL:
     lib.dspark_verify.restype = I
     lib.dspark_read_device_error.argtypes = [P, S, ctypes.POINTER(ctypes.c_uint32)]
     lib.dspark_read_device_error.restype = I
+    lib.dspark_schedule_static.argtypes = [P, P, P, I, I, I, P, P, P, P, S]
+    lib.dspark_schedule_static.restype = I
     lib.dspark_status_string.argtypes = [I]
     lib.dspark_status_string.restype = ctypes.c_char_p
     return lib
@@ -127,6 +129,21 @@ def dspark_schedule(conf_logits, temps, profile_ms, verify_len, survival, row_st
         _ptr(row_start, "row_start", torch.int64, B), _ptr(n_tokens, "n_tokens", torch.int32, 1),
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check("dspark_schedule", st)
+
+
+def dspark_schedule_static(conf_logits, temps, profile_ms, verify_len, survival, row_start, n_tokens,
+                           stream=None) -> None:
+    """dspark_schedule without a workspace (scratch in a static device array
+    inside the library), for callers that cannot allocate device memory. Same
+    outputs; B*K is limited to 16384; calls must not overlap on the GPU."""
+    B, K = conf_logits.shape
+    st = lib.dspark_schedule_static(
+        _ptr(conf_logits, "conf_logits", torch.float32), _ptr(temps, "temps", torch.float32, K),
+        _ptr(profile_ms, "profile_ms", torch.float32), profile_ms.numel(), B, K,
+        _ptr(verify_len, "verify_len", torch.int32, B), _ptr(survival, "survival", torch.float32, B * K),
+        _ptr(row_start, "row_start", torch.int64, B), _ptr(n_tokens, "n_tokens", torch.int32, 1),
+        _stream(stream))
+    _check("dspark_schedule_static", st)
 
 
 def dspark_verify(target_logits, row_start, z, lse_q, q_tok, draft_tokens, verify_len, u_accept, u_resample,
