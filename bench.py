@@ -57,7 +57,7 @@ class ClockSampler:
                0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period: float = 0.1):
+    def __init__(self, index: int, period: float = 0.02):
         self.samples, self.reasons, self.period = [], set(), period
         self.ok = False
         try:

@@ -158,6 +158,15 @@ dspark_status dspark_schedule_static(const float* conf_logits, const float* temp
                                      int32_t* verify_len, float* survival, int64_t* row_start,
                                      int32_t* n_tokens, dspark_stream_t stream);
 
+/* Ask the CUDA runtime to set aside up to `bytes` of the current device's L2
+ * for persisting accesses (cudaLimitPersistingL2CacheSize, capped at the
+ * device's maximum); *granted (if non-NULL) receives the size in effect. The
+ * draft kernel reads the Markov factor Bf with an L2 evict-last hint at every
+ * position, and such lines are only kept in this set-aside, which is empty by
+ * default. The setting belongs to the calling process's CUDA context and
+ * ends with it; call once at set-up, outside stream capture. */
+dspark_status dspark_l2_reserve(size_t bytes, size_t* granted);
+
 /* Synchronise `stream`, return the status recorded in the workspace's error
  * word (DSPARK_OK if none) and clear it; *detail (if non-NULL) receives the
  * offending value or the index of the wait that timed out. */

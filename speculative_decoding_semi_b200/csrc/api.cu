@@ -10,6 +10,9 @@
 namespace dspark {
 cudaError_t launch_draft_generic(DraftArgs a, int G, cudaStream_t stream);
 int draft_grid_size(int V, int sms);
+bool draft_tc_supported(const DraftArgs& a);
+int draft_tc_grid(int V, int sms);
+cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cudaStream_t stream);
 }  // namespace dspark
 
 using namespace dspark;
@@ -61,8 +64,6 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DSPARK_ERR_CUDA;
-  const int G = draft_grid_size(V, sms);
-
   DraftArgs a{};
   a.base = base_logits;
   a.A = A;
@@ -80,13 +81,20 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
   a.z = z;
   a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
   a.sync = reinterpret_cast<unsigned*>(ws + kSyncOffset);
+  // bf16 factors with r % 64 == 0 (r <= 256) and V % 32 == 0 take the
+  // tensor-core kernel; other shapes and fp32 factors the CUDA-core kernel
+  const bool tc = draft_tc_supported(a);
+  const int G = tc ? draft_tc_grid(V, sms) : draft_grid_size(V, sms);
   char* scratch = ws + kScratchOffset;
+  const size_t gmax = std::min<size_t>(kMaxGrid, V / 8);
   a.part_m = reinterpret_cast<float*>(scratch);
-  a.part_S = reinterpret_cast<double*>(scratch + align_up(static_cast<size_t>(B) * G * sizeof(float), 256));
+  a.part_S = reinterpret_cast<double*>(scratch + align_up(static_cast<size_t>(B) * gmax * sizeof(float), 256));
+  char* extra = scratch + align_up(static_cast<size_t>(B) * gmax * sizeof(float), 256) +
+                align_up(static_cast<size_t>(B) * gmax * sizeof(double), 256);
 
-  cudaError_t e = cudaMemsetAsync(a.sync, 0, 2u * K * sizeof(unsigned), s);
+  cudaError_t e = cudaMemsetAsync(a.sync, 0, kSyncBytes, s);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
-  return from_cuda(launch_draft_generic(a, G, s));
+  return from_cuda(tc ? launch_draft_tc(a, G, a.sync, extra, s) : launch_draft_generic(a, G, s));
 }
 
 dspark_status dspark_schedule(const float* conf_logits, const float* temps, const float* profile_ms,
@@ -146,6 +154,19 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
   a.n_out = n_out;
   a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
   return from_cuda(launch_verify(a, ws + kScratchOffset, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_l2_reserve(size_t bytes, size_t* granted) {
+  int dev = 0, max_persist = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev) != cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  const size_t want = std::min(bytes, static_cast<size_t>(max_persist));
+  if (cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, want) != cudaSuccess) return DSPARK_ERR_CUDA;
+  size_t now = 0;
+  if (cudaDeviceGetLimit(&now, cudaLimitPersistingL2CacheSize) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (granted) *granted = now;
+  return DSPARK_OK;
 }
 
 dspark_status dspark_read_device_error(void* workspace, dspark_stream_t stream, uint32_t* detail) {

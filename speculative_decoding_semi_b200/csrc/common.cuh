@@ -79,28 +79,26 @@ static __device__ __noinline__ bool wait_at_least(const unsigned* ctr, unsigned 
 
 // CTA-wide: thread 0 waits, the result is broadcast; all threads then see the
 // producers' writes (acquire by thread 0, ordered for the CTA by the barrier).
+template <class Sync>
 __device__ __forceinline__ bool cta_wait_at_least(const unsigned* ctr, unsigned target, unsigned* err,
-                                                  unsigned where, int* s_flag) {
-  if (threadIdx.x == 0) {
-    bool ok = wait_at_least(ctr, target, err, where);
-    __threadfence();
-    *s_flag = ok ? 1 : 0;
-  }
-  __syncthreads();
-  bool ok = *s_flag != 0;
-  __syncthreads();
-  return ok;
-}
+                                                  unsigned where, int* s_flag);
 
 // CTA-wide release: every thread's prior global writes become visible before
 // the counter moves.
-__device__ __forceinline__ void cta_release_add(unsigned* ctr, unsigned v) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    red_release_gpu_add(ctr, v);
-  }
-}
+template <class Sync>
+__device__ __forceinline__ void cta_release_add(unsigned* ctr, unsigned v);
+
+
+// ------------------------------------------------------ barrier policies
+// Whole-CTA barrier, or a named barrier over the first NT threads (used by
+// warp-specialised kernels whose other warps never join).
+struct CtaSync {
+  __device__ __forceinline__ static void sync() { __syncthreads(); }
+};
+template <int ID, int NT>
+struct NamedSync {
+  __device__ __forceinline__ static void sync() { asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(NT) : "memory"); }
+};
 
 // ----------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_max(float v) {
@@ -126,46 +124,46 @@ __device__ __forceinline__ int warp_max_int(int v) {
 
 // Block-wide reductions; `red` is shared scratch of >= 32 elements. All
 // threads of the block must call; every thread gets the result.
-template <int NT>
+template <int NT, class Sync = CtaSync>
 __device__ __forceinline__ float block_max(float v, float* red) {
   v = warp_max(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
+  Sync::sync();
   if (l == 0) red[w] = v;
-  __syncthreads();
+  Sync::sync();
   v = (l < NT / 32) ? red[l] : -INFINITY;
   v = warp_max(v);
   return v;
 }
-template <int NT>
+template <int NT, class Sync = CtaSync>
 __device__ __forceinline__ double block_sum(double v, double* red) {
   v = warp_sum(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
+  Sync::sync();
   if (l == 0) red[w] = v;
-  __syncthreads();
+  Sync::sync();
   v = (l < NT / 32) ? red[l] : 0.0;
   v = warp_sum(v);
   return v;
 }
-template <int NT>
+template <int NT, class Sync = CtaSync>
 __device__ __forceinline__ int block_min_int(int v, int* red) {
   v = warp_min_int(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
+  Sync::sync();
   if (l == 0) red[w] = v;
-  __syncthreads();
+  Sync::sync();
   v = (l < NT / 32) ? red[l] : 0x7fffffff;
   v = warp_min_int(v);
   return v;
 }
-template <int NT>
+template <int NT, class Sync = CtaSync>
 __device__ __forceinline__ int block_max_int(int v, int* red) {
   v = warp_max_int(v);
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();
+  Sync::sync();
   if (l == 0) red[w] = v;
-  __syncthreads();
+  Sync::sync();
   v = (l < NT / 32) ? red[l] : -0x7fffffff;
   v = warp_max_int(v);
   return v;
@@ -184,15 +182,15 @@ __device__ __forceinline__ double warp_inclusive_scan(double v) {
 
 // Block-wide exclusive scan of fp64 (thread order); returns the exclusive
 // prefix, writes the block total to *total. `red` >= 33 doubles of shared.
-template <int NT>
+template <int NT, class Sync = CtaSync>
 __device__ __forceinline__ double block_exclusive_scan(double v, double* red, double* total) {
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   double inc = warp_inclusive_scan(v);
   double exw = __shfl_up_sync(0xffffffffu, inc, 1);
   if (l == 0) exw = 0.0;
-  __syncthreads();
+  Sync::sync();
   if (l == 31) red[w] = inc;
-  __syncthreads();
+  Sync::sync();
   if (w == 0) {
     double s = (l < NT / 32) ? red[l] : 0.0;
     double si = warp_inclusive_scan(s);
@@ -201,11 +199,104 @@ __device__ __forceinline__ double block_exclusive_scan(double v, double* red, do
     if (l < NT / 32) red[l] = se;
     if (l == NT / 32 - 1) red[32] = si;
   }
-  __syncthreads();
+  Sync::sync();
   double ex = red[w] + exw;
   *total = red[32];
-  __syncthreads();
+  Sync::sync();
   return ex;
+}
+
+template <class Sync>
+__device__ __forceinline__ bool cta_wait_at_least(const unsigned* ctr, unsigned target, unsigned* err,
+                                                  unsigned where, int* s_flag) {
+  if (threadIdx.x == 0) {
+    bool ok = wait_at_least(ctr, target, err, where);
+    __threadfence();
+    *s_flag = ok ? 1 : 0;
+  }
+  Sync::sync();
+  bool ok = *s_flag != 0;
+  Sync::sync();
+  return ok;
+}
+
+template <class Sync>
+__device__ __forceinline__ void cta_release_add(unsigned* ctr, unsigned v) {
+  Sync::sync();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_gpu_add(ctr, v);
+  }
+}
+
+// One warp: the first element (vocabulary order) of a run of n elements
+// (n a multiple of 4) whose running fp64 sum of weights exceeds R, with a
+// positive weight; -1 if rounding leaves none (*last_pos then gives the last
+// positive one). Elements are read as coalesced rows of 128: lane l holds
+// elements 4l..4l+3 of each row, `load(e)` returns the data for elements
+// e..e+3 and `weigh(data, w)` their four weights. Up to kRows rows are loaded
+// at once into registers before scanning; longer runs go row by row.
+template <int kRows, class T, class Load, class Weigh>
+__device__ __forceinline__ int scan_rows128(int n, int lane, double R, Load load, Weigh weigh, int* last_pos) {
+  const int nrows = (n + 127) / 128;
+  double before = 0.0;
+  int found = -1, last = -1;
+  auto process = [&](int r0, const T& v) {
+    const int e = r0 + 4 * lane;
+    double w[4] = {0.0, 0.0, 0.0, 0.0};
+    if (e < n) weigh(v, w);
+    const double ls = ((w[0] + w[1]) + w[2]) + w[3];
+    double inc = ls;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double nb = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += nb;
+    }
+    double exc = __shfl_up_sync(0xffffffffu, inc, 1);
+    if (lane == 0) exc = 0.0;
+    const double ex_l = before + exc;
+    int hitc = -1;
+    if (e < n && ex_l + ls > R) {
+      double cc = ex_l;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (hitc < 0 && cc + w[c] > R && w[c] > 0.0) hitc = c;
+        cc += w[c];
+      }
+    }
+    const unsigned hits = __ballot_sync(0xffffffffu, hitc >= 0);
+    if (hits) {
+      const int hl = __ffs(hits) - 1;
+      found = r0 + 4 * hl + __shfl_sync(0xffffffffu, hitc, hl);
+    }
+    int lp = -1;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      if (e + c < n && w[c] > 0.0) lp = e + c;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lp = max(lp, __shfl_xor_sync(0xffffffffu, lp, o));
+    last = max(last, lp);
+    before += __shfl_sync(0xffffffffu, inc, 31);
+  };
+  if (nrows <= kRows) {
+    T buf[kRows];
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) {
+      const int e = j * 128 + 4 * lane;
+      if (j < nrows && e < n) buf[j] = load(e);
+    }
+#pragma unroll
+    for (int j = 0; j < kRows; ++j)
+      if (j < nrows && found < 0) process(j * 128, buf[j]);
+  } else {
+    for (int r0 = 0; r0 < n && found < 0; r0 += 128) {
+      T v;
+      if (r0 + 4 * lane < n) v = load(r0 + 4 * lane);
+      process(r0, v);
+    }
+  }
+  *last_pos = last;
+  return found;
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {

@@ -113,18 +113,18 @@ __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
       __syncthreads();
     }
     // ---- 2. every chunk of position i is in HBM
-    cta_release_add(&a.sync[2 * i], 1u);
+    cta_release_add<CtaSync>(&a.sync[2 * i], 1u);
     // ---- 3. select the tokens of my requests
     if (g < a.B) {
-      if (!cta_wait_at_least(&a.sync[2 * i], static_cast<unsigned>(G), a.err, 2u * i, &s_flag)) return;
+      if (!cta_wait_at_least<CtaSync>(&a.sync[2 * i], static_cast<unsigned>(G), a.err, 2u * i, &s_flag)) return;
       for (int b = g; b < a.B; b += G) {
-        select_token<DT>(a, b, i, G);
-        cta_release_add(&a.sync[2 * i + 1], 1u);
+        select_token<DT, CtaSync>(a, b, i, G, 8);
+        cta_release_add<CtaSync>(&a.sync[2 * i + 1], 1u);
       }
     }
     // ---- 4. all tokens of position i
     if (i + 1 < a.K) {
-      if (!cta_wait_at_least(&a.sync[2 * i + 1], static_cast<unsigned>(a.B), a.err, 2u * i + 1u, &s_flag))
+      if (!cta_wait_at_least<CtaSync>(&a.sync[2 * i + 1], static_cast<unsigned>(a.B), a.err, 2u * i + 1u, &s_flag))
         return;
     }
   }
@@ -132,14 +132,15 @@ __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
 
 }  // namespace
 
+size_t draft_tc_extra_bytes(int B, int V, int r);
+
 size_t draft_scratch_bytes(int B, int K, int V, int r) {
   (void)K;
-  (void)r;
   const size_t G = std::min<size_t>(kMaxGrid, V / 8);
   size_t off = 0;
   off = align_up(off + static_cast<size_t>(B) * G * sizeof(float), 256);
   off = align_up(off + static_cast<size_t>(B) * G * sizeof(double), 256);
-  return off;
+  return off + draft_tc_extra_bytes(B, V, r);
 }
 
 int draft_grid_size(int V, int sms) { return std::max(1, std::min(std::min(kMaxGrid, sms), V / 8)); }

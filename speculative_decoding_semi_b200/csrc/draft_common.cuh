@@ -20,72 +20,38 @@ __device__ __forceinline__ int previous_token(const DraftArgs& a, int b, int i) 
   return t;
 }
 
-// Inverse-CDF draw of request b at position i from the G chunk partials
-// (m_c, S_c = sum_{v in chunk c} exp(z_v - m_c)). Chunks are combined in
-// vocabulary order in fp64 with the common shift M = max m_c; the chunk whose
-// inclusive prefix first exceeds u*W is rescanned with weights exp(z - m_c) *
-// exp(m_c - M), and the first element whose running sum exceeds the remainder
-// is the token (strict '>', so a zero weight is never drawn). Writes
-// draft_tokens, q_tok = w_t / W and lse_q = M + log W. All NT threads call.
-template <int NT>
-__device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int G) {
-  __shared__ float redf[32];
+// Vocabulary chunk of CTA c when V is split into `unit`-wide pieces over G CTAs.
+__device__ __forceinline__ void chunk_bounds(int V, int unit, int G, int c, int* lo, int* hi) {
+  const int U = V / unit;
+  *lo = static_cast<int>(static_cast<long long>(c) * U / G) * unit;
+  *hi = static_cast<int>(static_cast<long long>(c + 1) * U / G) * unit;
+}
+
+// First element k of z[lo,hi) at which the running sum of exp(z_k - m) * f
+// exceeds R (strict '>'), with each thread scanning a contiguous stretch; if
+// rounding leaves no such element, the last one with a positive weight.
+// Returns the index (>= lo) to every thread.
+template <int NT, class Sync>
+__device__ __forceinline__ int rescan_range(const float* zrow, int lo, int hi, float m, double f, double R) {
   __shared__ double redd[33];
   __shared__ int redi[32];
-  __shared__ double s_W, s_exc;
   const int tid = threadIdx.x;
-  const long long pb = static_cast<long long>(b) * G;
-  float mc = -INFINITY;
-  double Sc = 0.0;
-  if (tid < G) {
-    mc = __ldcg(a.part_m + pb + tid);
-    Sc = __ldcg(a.part_S + pb + tid);
-  }
-  const float M = block_max<NT>(mc, redf);
-  const double wc = (tid < G) ? __dmul_rn(Sc, exp(static_cast<double>(mc) - static_cast<double>(M))) : 0.0;
-  double total;
-  const double ex = block_exclusive_scan<NT>(wc, redd, &total);
-  if (tid == G - 1) s_W = ex + wc;
-  __syncthreads();
-  const double W = s_W;
-  const long long zrow = (static_cast<long long>(b) * a.K + i) * a.V;
-  if (!(W > 0.0) || !(W < INFINITY)) {  // non-finite logits
-    if (tid == 0) {
-      set_error(a.err, DSPARK_ERR_DEVICE_ASSERT, 0x30000000u | static_cast<unsigned>(b));
-      a.tokens[static_cast<long long>(b) * a.K + i] = 0;
-      a.q_tok[static_cast<long long>(b) * a.K + i] = 0.f;
-      a.lse_q[static_cast<long long>(b) * a.K + i] = 0.0;
-    }
-    __syncthreads();
-    return;
-  }
-  const double thr = static_cast<double>(a.u[static_cast<long long>(b) * a.K + i]) * W;
-  int c = block_min_int<NT>((tid < G && ex + wc > thr) ? tid : 0x7fffffff, redi);
-  if (c == 0x7fffffff) c = G - 1;
-  if (tid == c) s_exc = ex;
-  __syncthreads();
-  const double R = thr - s_exc;
-  const int NU = a.V / 8;
-  const int lo = static_cast<int>(static_cast<long long>(c) * NU / G) * 8;
-  const int hi = static_cast<int>(static_cast<long long>(c + 1) * NU / G) * 8;
-  const float m_c = __ldcg(a.part_m + pb + c);
-  const double f_c = exp(static_cast<double>(m_c) - static_cast<double>(M));
   const int per = (hi - lo + NT - 1) / NT;
   const int e_lo = min(hi, lo + tid * per), e_hi = min(hi, e_lo + per);
   double lw = 0.0;
   int last_pos = -1;
   for (int k = e_lo; k < e_hi; ++k) {
-    const double w = __dmul_rn(static_cast<double>(expf(__ldcg(a.z + zrow + k) - m_c)), f_c);
+    const double w = __dmul_rn(static_cast<double>(expf(__ldcg(zrow + k) - m)), f);
     lw += w;
     if (w > 0.0) last_pos = k;
   }
-  double tot2;
-  const double ex2 = block_exclusive_scan<NT>(lw, redd, &tot2);
+  double tot;
+  const double ex = block_exclusive_scan<NT, Sync>(lw, redd, &tot);
   int found = 0x7fffffff;
-  if (e_lo < e_hi && ex2 + lw > R) {
-    double cum = ex2;
+  if (e_lo < e_hi && ex + lw > R) {
+    double cum = ex;
     for (int k = e_lo; k < e_hi; ++k) {
-      const double w = __dmul_rn(static_cast<double>(expf(__ldcg(a.z + zrow + k) - m_c)), f_c);
+      const double w = __dmul_rn(static_cast<double>(expf(__ldcg(zrow + k) - m)), f);
       cum += w;
       if (cum > R && w > 0.0) {
         found = k;
@@ -94,17 +60,106 @@ __device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int 
     }
     if (found == 0x7fffffff && last_pos >= 0) found = last_pos;
   }
-  int t = block_min_int<NT>(found, redi);
-  if (t == 0x7fffffff) t = block_max_int<NT>(last_pos, redi);
+  int t = block_min_int<NT, Sync>(found, redi);
+  if (t == 0x7fffffff) t = block_max_int<NT, Sync>(last_pos, redi);
+  return max(t, lo);
+}
+
+// Inverse-CDF draw of request b at position i from the G chunk partials
+// (m_c, S_c = sum_{v in chunk c} exp(z_v - m_c)); chunk c covers the
+// vocabulary slice chunk_bounds(V, unit, G, c). The chunks are combined in
+// vocabulary order in fp64 with the common shift M = max m_c; the chunk whose
+// inclusive prefix first exceeds u*W is rescanned with the same weights
+// exp(z - m_c) * exp(m_c - M) (bit-identical to the ones summed when m_c is
+// the shift used by the producer), and the first element whose running sum
+// exceeds the remainder is the token (strict '>', so a zero weight is never
+// drawn). If W is not a normal positive number (the producer's shift left
+// every weight underflowing or some overflowing), the row is redone with its
+// exact maximum as the shift. Writes draft_tokens, q_tok = w_t / W and
+// lse_q = M + log W. All NT threads call.
+template <int NT, class Sync>
+__device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int G, int unit) {
+  __shared__ float redf[32];
+  __shared__ double redd[33];
+  __shared__ int redi[32];
+  __shared__ double s_W, s_exc;
+  const int tid = threadIdx.x;
+  const long long pb = static_cast<long long>(b) * G;
+  const long long o = static_cast<long long>(b) * a.K + i;
+  const float* zrow = a.z + o * a.V;
+  float mc = -INFINITY;
+  double Sc = 0.0;
+  if (tid < G) {
+    mc = __ldcg(a.part_m + pb + tid);
+    Sc = __ldcg(a.part_S + pb + tid);
+  }
+  float M = block_max<NT, Sync>(mc, redf);
+  const double wc = (tid < G) ? __dmul_rn(Sc, exp(static_cast<double>(mc) - static_cast<double>(M))) : 0.0;
+  double total;
+  const double ex = block_exclusive_scan<NT, Sync>(wc, redd, &total);
+  if (tid == G - 1) s_W = ex + wc;
+  Sync::sync();
+  double W = s_W;
+  const double u = static_cast<double>(a.u[o]);
+  int t;
+  float m_t;
+  double f_t;
+  if (W >= 1e-30 && W <= 1e30) {
+    const double thr = u * W;
+    int c = block_min_int<NT, Sync>((tid < G && ex + wc > thr) ? tid : 0x7fffffff, redi);
+    if (c == 0x7fffffff) c = G - 1;
+    if (tid == c) s_exc = ex;
+    Sync::sync();
+    const double R = thr - s_exc;
+    int lo, hi;
+    chunk_bounds(a.V, unit, G, c, &lo, &hi);
+    m_t = __ldcg(a.part_m + pb + c);
+    f_t = exp(static_cast<double>(m_t) - static_cast<double>(M));
+    t = rescan_range<NT, Sync>(zrow, lo, hi, m_t, f_t, R);
+  } else {
+    // whole row with its exact maximum as the shift
+    float mx = -INFINITY;
+    for (int k = tid; k < a.V; k += NT) mx = fmaxf(mx, __ldcg(zrow + k));
+    M = block_max<NT, Sync>(mx, redf);
+    double s = 0.0;
+    for (int k = tid; k < a.V; k += NT) s += static_cast<double>(expf(__ldcg(zrow + k) - M));
+    W = block_sum<NT, Sync>(s, redd);
+    if (!(W > 0.0) || !(W < INFINITY)) {  // non-finite logits
+      if (tid == 0) {
+        set_error(a.err, DSPARK_ERR_DEVICE_ASSERT, 0x30000000u | static_cast<unsigned>(b));
+        a.tokens[o] = 0;
+        a.q_tok[o] = 0.f;
+        a.lse_q[o] = 0.0;
+      }
+      Sync::sync();
+      return;
+    }
+    m_t = M;
+    f_t = 1.0;
+    // the rescan's own running total is the W that u scales
+    double Wscan;
+    {
+      const int per = (a.V + NT - 1) / NT;
+      const int e_lo = min(a.V, tid * per), e_hi = min(a.V, e_lo + per);
+      double lw = 0.0;
+      for (int k = e_lo; k < e_hi; ++k) lw += static_cast<double>(expf(__ldcg(zrow + k) - M));
+      double tot;
+      const double exs = block_exclusive_scan<NT, Sync>(lw, redd, &tot);
+      if (e_hi == a.V && e_lo < e_hi) s_W = exs + lw;
+      Sync::sync();
+      Wscan = s_W;
+      Sync::sync();
+    }
+    W = Wscan;
+    t = rescan_range<NT, Sync>(zrow, 0, a.V, M, 1.0, u * W);
+  }
   if (tid == 0) {
-    t = max(t, lo);
-    const double w_t = __dmul_rn(static_cast<double>(expf(__ldcg(a.z + zrow + t) - m_c)), f_c);
-    const long long o = static_cast<long long>(b) * a.K + i;
+    const double w_t = __dmul_rn(static_cast<double>(expf(__ldcg(zrow + t) - m_t)), f_t);
     a.tokens[o] = t;
     a.q_tok[o] = static_cast<float>(w_t / W);
     a.lse_q[o] = static_cast<double>(M) + log(W);
   }
-  __syncthreads();
+  Sync::sync();
 }
 
 }  // namespace dspark

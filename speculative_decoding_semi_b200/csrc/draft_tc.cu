@@ -1,0 +1,897 @@
+// Semi-autoregressive Markov draft on the 5th-generation tensor cores.
+//
+// QbitAI article "DSpark: ten concepts are enough", sections "DSpark = Eagle +
+// DFlash" and "a cheaper sequential module: the Markov head": base logits from
+// the parallel backbone are corrected left to right by a rank-256 bias that
+// depends only on the previous token. Here the bias of a group of requests at
+// position i is one GEMM, bias[v, b] = sum_k Bf[k, v] * A[t_b, k], run on
+// tcgen05 with the accumulator in TMEM and fused with the logit correction,
+// the write of z and the fp64 sums the inverse-CDF draw needs.
+//
+// One persistent cooperative kernel, one CTA per SM; CTA g owns the vocabulary
+// slice chunk_bounds(V, 32, G, g) for every request. Requests are split into
+// groups (of up to 128) that synchronise independently, so while one group's
+// tokens are being drawn the CTA streams another group's logits. Warp roles:
+//   warps 0-7  epilogue: read the accumulator (warp w reads TMEM lanes
+//              32*(w%4).. = vocabulary rows; columns = requests), add the base
+//              logits staged by TMA, write z back through TMA, and sum exp(z)
+//              in fp64 per request over the CTA's slice;
+//   warp 8     TMA producer of Bf tiles (ring of stages, L2 evict-last so the
+//              78 MB factor can stay resident across positions);
+//   warp 9     TMEM owner and MMA issuer (M = 128 vocabulary rows, N = the
+//              group's requests, K = r in steps of 16); it bulk-loads each
+//              group's operand (the A rows of the last drawn tokens, already
+//              in MMA layout) once the group's tokens are published;
+//   warp 10    selector: publishes the slice sums, waits for every CTA, draws
+//              the tokens of its requests (b mod G == g) by a two-level
+//              inverse-CDF search (the G slice sums, then the chosen slice's z),
+//              writes the A rows of the drawn tokens into the operand image and
+//              waits for the group's tokens before releasing the next position.
+// The epilogue streams base and z through per-warp TMA rings (L2 evict-first)
+// that run ahead across positions, since they do not depend on the tokens.
+// The exponentials use a fixed shift of 0, so each weight is exp(z) itself and
+// both levels of the search sum the same fp32 weights in fp64; a row whose
+// sum leaves [1e-30, 1e30] is redone by the selector with its exact maximum.
+// Every wait is bounded and reports DSPARK_ERR_TIMEOUT.
+#include <algorithm>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "draft_common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace dspark {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kEpiWarps = 8;
+constexpr int kProdWarp = kEpiWarps;
+constexpr int kMmaWarp = kEpiWarps + 1;
+constexpr int kSelWarp = kEpiWarps + 2;
+constexpr int kThreads = (kEpiWarps + 3) * 32;
+constexpr int kUnit = 32;                       // vocabulary granularity (one TMEM lane quadrant)
+constexpr int kTileRows = 128;                  // MMA M
+constexpr int kKStage = 64;                     // r per Bf stage (one 128-byte swizzle atom)
+constexpr int kMaxBfStages = 8;
+constexpr int kBfBoxBytes = 64 * kKStage * 2;   // 64 vocabulary x 64 r, bf16
+constexpr int kBfStageBytes = 2 * kBfBoxBytes;  // a 128-row tile
+constexpr int kChunk = 32;                      // requests per TMEM load and per z box
+constexpr int kBoxBytes = kChunk * kUnit * 4;   // 32 requests x 32 vocabulary, fp32
+constexpr int kMaxGroup = 128;                  // requests per MMA (N)
+constexpr int kMaxGroups = 4;                   // so B <= 512 on this path
+constexpr int kMaxRingSlots = 8;
+constexpr int kMaxAccSlots = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kBarBytes = 1024;
+
+struct TcParams {
+  DraftArgs d;
+  uint8_t* image;       // [groups][image_stride] A rows of the drawn tokens, MMA layout
+  unsigned* sync_part;  // [K][groups] slice sums published
+  unsigned* sync_tok;   // [K+1][groups] tokens and operand rows published ([0]: anchors)
+  int gsize;            // requests per group (multiple of 16, <= 128)
+  int ngroups;
+  int r_stages;         // r / 64
+  int slot_stride;      // TMEM columns per accumulator slot
+  int nslots;
+  int nbf;              // Bf ring stages
+  int nbs;              // base/z ring slots per epilogue warp
+  int image_stride;     // bytes per group in the operand image (and in shared memory)
+};
+
+struct Layout {
+  int bf, brows, ring, part, bar, misc, total;
+};
+
+__host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs, int part_bytes) {
+  Layout L;
+  L.bf = 0;
+  L.brows = L.bf + nbf * kBfStageBytes;
+  L.ring = L.brows + ((brows_bytes + 1023) / 1024) * 1024;
+  L.part = L.ring + kEpiWarps * nbs * kBoxBytes;
+  L.bar = L.part + ((part_bytes + 15) / 16) * 16;
+  L.misc = L.bar + kBarBytes;
+  L.total = L.misc + 64;
+  return L;
+}
+
+struct Bars {
+  uint64_t* bf_full;       // [kMaxBfStages]
+  uint64_t* bf_empty;      // [kMaxBfStages]
+  uint64_t* acc_full;      // [kMaxAccSlots]
+  uint64_t* acc_empty;     // [kMaxAccSlots]
+  uint64_t* brows_full;
+  uint64_t* mma_done;
+  uint64_t* final_mma;
+  uint64_t* tokens_ready;  // [kMaxGroups]
+  uint64_t* step_done;     // [kMaxGroups]
+  uint64_t* base_full;     // [kEpiWarps][kMaxRingSlots]
+};
+
+__device__ __forceinline__ Bars carve_bars(uint8_t* p) {
+  Bars b;
+  uint64_t* q = reinterpret_cast<uint64_t*>(p);
+  b.bf_full = q;
+  q += kMaxBfStages;
+  b.bf_empty = q;
+  q += kMaxBfStages;
+  b.acc_full = q;
+  q += kMaxAccSlots;
+  b.acc_empty = q;
+  q += kMaxAccSlots;
+  b.brows_full = q++;
+  b.mma_done = q++;
+  b.final_mma = q++;
+  b.tokens_ready = q;
+  q += kMaxGroups;
+  b.step_done = q;
+  q += kMaxGroups;
+  b.base_full = q;
+  return b;
+}
+
+__device__ __forceinline__ int group_real(const TcParams& p, int gr) { return min(p.gsize, p.d.B - gr * p.gsize); }
+__device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
+// chunks c (32 requests each) with c % 2 == h among the group's real columns
+__device__ __forceinline__ int chunks_for(int ncol, int h) {
+  const int nch = (ncol + kChunk - 1) / kChunk;
+  return nch > h ? (nch - h + 1) / 2 : 0;
+}
+
+// Tile visited t-th in pass (i, gr): passes over the slice alternate
+// direction, so each pass starts on the Bf tiles the previous one touched last
+// (the ones most likely still in L2).
+__device__ __forceinline__ int phys_tile(int i, int gr, int ngroups, int ntiles, int t) {
+  return ((i * ngroups + gr) & 1) ? ntiles - 1 - t : t;
+}
+
+// The sequence of (position, group, tile, chunk) boxes one epilogue warp
+// streams, in consumption order; the TMA refill cursor walks it ahead of the
+// consumer across positions.
+struct Items {
+  const TcParams* p;
+  int ntiles, last_rows, q, h;
+  int i, gr, t, k;
+  bool valid;
+  __device__ int ptile() const { return phys_tile(i, gr, p->ngroups, ntiles, t); }
+  __device__ bool tile_ok() const { return kUnit * q < (ptile() == ntiles - 1 ? last_rows : kTileRows); }
+  __device__ void normalize() {
+    while (valid) {
+      if (i >= p->d.K) {
+        valid = false;
+        break;
+      }
+      if (gr >= p->ngroups) {
+        gr = 0;
+        ++i;
+        continue;
+      }
+      if (t >= ntiles) {
+        t = 0;
+        ++gr;
+        continue;
+      }
+      if (!tile_ok() || k >= chunks_for(group_real(*p, gr), h)) {
+        k = 0;
+        ++t;
+        continue;
+      }
+      break;
+    }
+  }
+  __device__ void first() {
+    i = gr = t = k = 0;
+    valid = true;
+    normalize();
+  }
+  __device__ void next() {
+    ++k;
+    normalize();
+  }
+};
+
+// Reduce 16 fp64 values across the 32 lanes of a warp by recursive halving:
+// afterwards lanes 2m and 2m+1 both hold the warp-wide sum of value m.
+__device__ __forceinline__ double reduce16(double (&w)[16], int lane) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const bool up = lane & 16;
+    const double send = up ? w[j] : w[j + 8];
+    const double keep = up ? w[j + 8] : w[j];
+    w[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const bool up = lane & 8;
+    const double send = up ? w[j] : w[j + 4];
+    const double keep = up ? w[j + 4] : w[j];
+    w[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const bool up = lane & 4;
+    const double send = up ? w[j] : w[j + 2];
+    const double keep = up ? w[j + 2] : w[j];
+    w[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  {
+    const bool up = lane & 2;
+    const double send = up ? w[0] : w[1];
+    const double keep = up ? w[1] : w[0];
+    w[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  return w[0] + __shfl_xor_sync(0xffffffffu, w[0], 1);
+}
+
+// Among n values x(0..n-1) (read through `get`) laid out in lane-contiguous
+// blocks, find the first index whose inclusive prefix exceeds `thr(total)`
+// (strict, never a zero entry); returns it, or the last positive index if
+// rounding leaves none, with its exclusive prefix in *excl and the sum of all
+// n values in *total. `thr` maps the total to the threshold, so one pass both
+// sums and searches. Sums run sequentially within a lane's block and in lane
+// order across blocks. One warp, all lanes; each lane's loads are issued
+// together (up to kSearchRegs values per lane stay in registers).
+template <int kSearchRegs, class Get, class Thr>
+__device__ __forceinline__ int warp_search(int n, Get get, Thr thr_of, int lane, double* excl, double* total) {
+  const int per = (n + 31) / 32;
+  const int lo = min(n, lane * per), hi = min(n, lo + per);
+  double local = 0.0;
+  int last_pos = -1;
+  double vals[kSearchRegs];
+  const bool in_regs = per <= kSearchRegs;
+  if (in_regs) {
+#pragma unroll
+    for (int j = 0; j < kSearchRegs; ++j) vals[j] = (lo + j < hi) ? get(lo + j) : 0.0;
+#pragma unroll
+    for (int j = 0; j < kSearchRegs; ++j) {
+      local += vals[j];
+      if (vals[j] > 0.0) last_pos = lo + j;
+    }
+  } else {
+    for (int x = lo; x < hi; ++x) {
+      const double v = get(x);
+      local += v;
+      if (v > 0.0) last_pos = x;
+    }
+  }
+  double inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double nb = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += nb;
+  }
+  double mine = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) mine = 0.0;
+  *total = __shfl_sync(0xffffffffu, inc, 31);
+  const double thr = thr_of(*total);
+  int found = 0x7fffffff;
+  double found_ex = 0.0;
+  if (lo < hi && mine + local > thr) {
+    double c = mine;
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kSearchRegs; ++j) {
+        if (found == 0x7fffffff && lo + j < hi) {
+          if (c + vals[j] > thr && vals[j] > 0.0) {
+            found = lo + j;
+            found_ex = c;
+          }
+          c += vals[j];
+        }
+      }
+    } else {
+      for (int x = lo; x < hi; ++x) {
+        const double v = get(x);
+        if (c + v > thr && v > 0.0) {
+          found = x;
+          found_ex = c;
+          break;
+        }
+        c += v;
+      }
+    }
+  }
+  int best = found;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if (best == 0x7fffffff) {
+    // rounding: the last positive entry, with its exclusive prefix from its owner
+    int lp = last_pos;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lp = max(lp, __shfl_xor_sync(0xffffffffu, lp, o));
+    best = max(lp, 0);
+    double e = 0.0;
+    if (best >= lo && best < hi) {
+      e = mine;
+      for (int x = lo; x < best; ++x) e += get(x);
+    }
+    const int owner = per > 0 ? min(31, best / per) : 0;
+    *excl = __shfl_sync(0xffffffffu, e, owner);
+    return best;
+  }
+  const int owner = per > 0 ? min(31, best / per) : 0;
+  *excl = __shfl_sync(0xffffffffu, found_ex, owner);
+  return best;
+}
+
+// Draw request b's token at position i (one warp). Writes draft_tokens,
+// q_tok and lse_q; returns the token.
+__device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane) {
+  const DraftArgs& d = p.d;
+  const long long o = static_cast<long long>(b) * d.K + i;
+  const float* zrow = d.z + o * d.V;
+  const double u = static_cast<double>(d.u[o]);
+  const double* part = d.part_S + static_cast<long long>(b) * G;
+  double ex, W;
+  // level 1: slice sums; their total is the W that u scales
+  const int c = warp_search<8>(
+      G, [&](int cc) { return __ldcg(part + cc); },
+      [&](double tot) { return (tot >= 1e-30 && tot <= 1e30) ? u * tot : INFINITY; }, lane, &ex, &W);
+  int tok;
+  double w_t;
+  float shift = 0.f;
+  if (W >= 1e-30 && W <= 1e30) {
+    const double R = u * W - ex;
+    // level 2: the slice's own weights exp(z), read as coalesced rows of 128
+    // (lane l holds elements 4l..4l+3 of each row) and scanned in vocabulary
+    // order: rows in turn, lanes in turn, then the lane's four elements
+    int lo, hi, x, last;
+    chunk_bounds(d.V, kUnit, G, c, &lo, &hi);
+    const int n = hi - lo;
+    const float* zc = zrow + lo;
+    x = scan_rows128<12, float4>(
+        n, lane, R, [&](int e) { return __ldcg(reinterpret_cast<const float4*>(zc + e)); },
+        [&](const float4& v, double(&w)[4]) {
+          w[0] = static_cast<double>(expf(v.x));
+          w[1] = static_cast<double>(expf(v.y));
+          w[2] = static_cast<double>(expf(v.z));
+          w[3] = static_cast<double>(expf(v.w));
+        },
+        &last);
+    if (x < 0) x = max(last, 0);  // rounding: the last positive weight
+    tok = lo + x;
+    w_t = static_cast<double>(expf(__ldcg(zc + x)));
+  } else {
+    // the whole row with its exact maximum as the shift
+    float mx = -INFINITY;
+    for (int k = lane; k < d.V; k += 32) mx = fmaxf(mx, __ldcg(zrow + k));
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+    shift = mx;
+    auto wz = [&](int k) { return static_cast<double>(expf(__ldcg(zrow + k) - mx)); };
+    tok = warp_search<8>(d.V, wz, [&](double tot) { return u * tot; }, lane, &ex, &W);
+    if (!(W > 0.0) || !(W < INFINITY)) {
+      if (lane == 0) set_error(d.err, DSPARK_ERR_DEVICE_ASSERT, 0x30000000u | static_cast<unsigned>(b));
+      tok = 0;
+      w_t = 0.0;
+      W = 1.0;
+    } else {
+      w_t = wz(tok);
+    }
+  }
+  if (lane == 0) {
+    d.tokens[o] = tok;
+    d.q_tok[o] = static_cast<float>(w_t / W);
+    d.lse_q[o] = static_cast<double>(shift) + log(W);
+  }
+  return tok;
+}
+
+// A row of the MMA's B operand for request b: A[t, :] into the operand image
+// of b's group, K-major with the 128-byte swizzle (one warp).
+__device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t, int lane) {
+  const int gr = b / p.gsize, n = b - gr * p.gsize;
+  const int N = round16(group_real(p, gr));
+  const int cpr = p.d.r / 8;
+  const uint4* A4 = reinterpret_cast<const uint4*>(p.d.A) + static_cast<long long>(t) * cpr;
+  uint8_t* img = p.image + static_cast<long long>(gr) * p.image_stride;
+  for (int ch = lane; ch < cpr; ch += 32) {
+    const uint4 v = __ldg(A4 + ch);
+    const int kb = ch >> 3, c = ch & 7;
+    *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) = v;
+  }
+}
+
+// One warp: lane 0 waits for *ctr >= target (bounded); the result goes to all lanes.
+__device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned target, unsigned* err,
+                                                  unsigned where, volatile int* abort, int lane) {
+  int ok = 1;
+  if (lane == 0) {
+    ok = wait_at_least(ctr, target, err, where) ? 1 : 0;
+    __threadfence();
+    if (!ok) *abort = 1;
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    draft_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_bf,
+                    const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_z) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const DraftArgs& d = p.d;
+  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, p.ngroups * 4 * p.gsize * 8);
+  Bars bars = carve_bars(smem + Ly.bar);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
+  double* s_part = reinterpret_cast<double*>(smem + Ly.part);  // [group][quadrant][gsize]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, g = blockIdx.x;
+  int lo, hi;
+  chunk_bounds(d.V, kUnit, G, g, &lo, &hi);
+  const int ntiles = (hi - lo + kTileRows - 1) / kTileRows;
+  const int last_rows = (hi - lo) - (ntiles - 1) * kTileRows;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kMaxBfStages; ++s) {
+      mbar_init(&bars.bf_full[s], 1);
+      mbar_init(&bars.bf_empty[s], 1);
+    }
+    for (int s = 0; s < kMaxAccSlots; ++s) {
+      mbar_init(&bars.acc_full[s], 1);
+      mbar_init(&bars.acc_empty[s], kEpiWarps);
+    }
+    mbar_init(bars.brows_full, 1);
+    mbar_init(bars.mma_done, 1);
+    mbar_init(bars.final_mma, 1);
+    for (int s = 0; s < kMaxGroups; ++s) {
+      mbar_init(&bars.tokens_ready[s], 1);
+      mbar_init(&bars.step_done[s], kEpiWarps);
+    }
+    for (int s = 0; s < kEpiWarps * kMaxRingSlots; ++s) mbar_init(&bars.base_full[s], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == kProdWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_bf);
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_parity[kMaxBfStages];
+      bool issued[kMaxBfStages];
+      for (int s = 0; s < kMaxBfStages; ++s) issued[s] = false;
+      bool ok = true;
+      for (int i = 0; ok && i < d.K; ++i)
+        for (int gr = 0; ok && gr < p.ngroups; ++gr)
+          for (int t = 0; ok && t < ntiles; ++t)
+            for (int s = 0; s < p.r_stages; ++s) {
+              if (!mbar_wait(&bars.bf_empty[stage], phase ^ 1u, s_abort, d.err, 0x100u)) {
+                ok = false;
+                break;
+              }
+              uint8_t* dst = smem + Ly.bf + stage * kBfStageBytes;
+              const int v0 = lo + phys_tile(i, gr, p.ngroups, ntiles, t) * kTileRows;
+              mbar_arrive_expect_tx(&bars.bf_full[stage], kBfStageBytes);
+              tma_load_2d(dst, &tm_bf, v0, s * kKStage, &bars.bf_full[stage], pol);
+              tma_load_2d(dst + kBfBoxBytes, &tm_bf, v0 + 64, s * kKStage, &bars.bf_full[stage], pol);
+              issued[stage] = true;
+              issued_parity[stage] = phase;
+              if (++stage == p.nbf) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+      // every load lands before the CTA can exit
+      for (int s = 0; s < p.nbf; ++s)
+        if (issued[s]) mbar_drain(&bars.bf_full[s], issued_parity[s], d.err, 0x101u);
+    }
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int stage = 0, slot = 0;
+      uint32_t phase = 0, slot_phase = 0, brows_phase = 0, done_phase = 0;
+      uint32_t tr_phase[kMaxGroups] = {0, 0, 0, 0};
+      bool brows_used = false;
+      const uint32_t brows_addr = smem_u32(smem + Ly.brows);
+      const uint32_t bf_addr = smem_u32(smem + Ly.bf);
+      bool ok = true;
+      for (int i = 0; ok && i < d.K; ++i)
+        for (int gr = 0; ok && gr < p.ngroups; ++gr) {
+          const int N = round16(group_real(p, gr));
+          const uint32_t idesc = idesc_bf16_f32(N, 1);
+          // the operand buffer is free once the previous group's MMAs are done
+          if (brows_used) {
+            mma_commit(bars.mma_done);
+            if (!mbar_wait(bars.mma_done, done_phase, s_abort, d.err, 0x204u)) {
+              ok = false;
+              break;
+            }
+            done_phase ^= 1u;
+          }
+          if (!mbar_wait(&bars.tokens_ready[gr], tr_phase[gr], s_abort, d.err, 0x200u)) {
+            ok = false;
+            break;
+          }
+          tr_phase[gr] ^= 1u;
+          fence_proxy_async_all();
+          const uint32_t bytes = static_cast<uint32_t>(N * d.r * 2);
+          mbar_arrive_expect_tx(bars.brows_full, bytes);
+          bulk_load(smem + Ly.brows, p.image + static_cast<long long>(gr) * p.image_stride, bytes,
+                    bars.brows_full);
+          if (!mbar_wait(bars.brows_full, brows_phase, s_abort, d.err, 0x205u)) {
+            ok = false;
+            break;
+          }
+          brows_phase ^= 1u;
+          brows_used = true;
+          tc_fence_after();
+          for (int t = 0; ok && t < ntiles; ++t) {
+            if (!mbar_wait(&bars.acc_empty[slot], slot_phase ^ 1u, s_abort, d.err, 0x201u)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t dcol = tmem_base + static_cast<uint32_t>(slot * p.slot_stride);
+            for (int s = 0; s < p.r_stages; ++s) {
+              if (!mbar_wait(&bars.bf_full[stage], phase, s_abort, d.err, 0x202u)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t a_base = bf_addr + stage * kBfStageBytes;
+              const uint32_t b_base = brows_addr + s * (N * 128);
+#pragma unroll
+              for (int kk = 0; kk < kKStage / 16; ++kk) {
+                const uint64_t adesc = smem_desc_sw128(a_base + kk * 2048, kBfBoxBytes, 1024);
+                const uint64_t bdesc = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                mma_bf16(dcol, adesc, bdesc, idesc, (s | kk) != 0);
+              }
+              mma_commit(&bars.bf_empty[stage]);
+              if (++stage == p.nbf) {
+                stage = 0;
+                phase ^= 1u;
+              }
+            }
+            if (!ok) break;
+            mma_commit(&bars.acc_full[slot]);
+            if (++slot == p.nslots) {
+              slot = 0;
+              slot_phase ^= 1u;
+            }
+          }
+        }
+      // all issued MMAs complete before TMEM is released
+      mma_commit(bars.final_mma);
+      mbar_drain(bars.final_mma, 0, d.err, 0x203u);
+    }
+  } else if (warp == kSelWarp) {
+    // ------------------------------------------------------------ selector
+    bool ok = true;
+    // position 0's operand: the anchors' rows, and zeros in padded rows
+    for (int b = g; b < d.B; b += G) write_image_row(p, b, previous_token(d, b, 0), lane);
+    if (g == 0) {
+      for (int gr = 0; gr < p.ngroups; ++gr) {
+        const int nreal = group_real(p, gr), N = round16(nreal);
+        uint8_t* img = p.image + static_cast<long long>(gr) * p.image_stride;
+        for (int n = nreal; n < N; ++n)
+          for (int ch = lane; ch < d.r / 8; ch += 32) {
+            const int kb = ch >> 3, c = ch & 7;
+            *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
+                make_uint4(0, 0, 0, 0);
+          }
+      }
+    }
+    __threadfence();
+    __syncwarp();
+    for (int gr = 0; gr < p.ngroups; ++gr) {
+      const int gbase = gr * p.gsize, nreal = group_real(p, gr);
+      unsigned mine = 0;
+      for (int b = g; b < d.B; b += G) mine += (b >= gbase && b < gbase + nreal) ? 1u : 0u;
+      if (lane == 0 && mine) red_release_gpu_add(&p.sync_tok[gr], mine);
+    }
+    for (int gr = 0; ok && gr < p.ngroups; ++gr) {
+      ok = warp_wait_counter(&p.sync_tok[gr], static_cast<unsigned>(group_real(p, gr)), d.err, 0x400u + gr,
+                             s_abort, lane);
+      if (ok && lane == 0) mbar_arrive(&bars.tokens_ready[gr]);
+    }
+    for (int i = 0; ok && i < d.K; ++i) {
+      for (int gr = 0; ok && gr < p.ngroups; ++gr) {
+        const int gbase = gr * p.gsize, nreal = group_real(p, gr);
+        if (!mbar_wait(&bars.step_done[gr], i & 1, s_abort, d.err, 0x500u)) {
+          ok = false;
+          break;
+        }
+        // this CTA's slice sums, summed over the four quadrants in a fixed order
+        const double* sp = s_part + gr * 4 * p.gsize;
+        for (int n = lane; n < nreal; n += 32) {
+          const double S = sp[n] + sp[p.gsize + n] + sp[2 * p.gsize + n] + sp[3 * p.gsize + n];
+          d.part_S[static_cast<long long>(gbase + n) * G + g] = S;
+          d.part_m[static_cast<long long>(gbase + n) * G + g] = 0.f;
+        }
+        __threadfence();
+        __syncwarp();
+        const unsigned slot = static_cast<unsigned>(i * p.ngroups + gr);
+        if (lane == 0) red_release_gpu_add(&p.sync_part[slot], 1u);
+        unsigned mine = 0;
+        // first request of this group drawn by CTA g: the smallest b >= gbase with b % G == g
+        const int first = gbase + ((g - gbase) % G + G) % G;
+        if (first < gbase + nreal) {
+          ok = warp_wait_counter(&p.sync_part[slot], static_cast<unsigned>(G), d.err, 0x600u + slot, s_abort, lane);
+          if (!ok) break;
+          for (int b = first; b < gbase + nreal; b += G) {
+            const int t = select_warp(p, b, i, G, lane);
+            if (i + 1 < d.K) write_image_row(p, b, t, lane);
+            ++mine;
+          }
+        }
+        if (i + 1 < d.K) {
+          const unsigned nslot = static_cast<unsigned>((i + 1) * p.ngroups + gr);
+          __threadfence();
+          __syncwarp();
+          if (lane == 0 && mine) red_release_gpu_add(&p.sync_tok[nslot], mine);
+          ok = warp_wait_counter(&p.sync_tok[nslot], static_cast<unsigned>(nreal), d.err, 0x700u + nslot, s_abort,
+                                 lane);
+          if (ok && lane == 0) mbar_arrive(&bars.tokens_ready[gr]);
+        }
+      }
+    }
+    if (!ok) *s_abort = 1;
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3, h = warp >> 2;
+    const uint64_t pol_first = policy_evict_first();
+    if (lane == 0) {
+      prefetch_tmap(&tm_base);
+      prefetch_tmap(&tm_z);
+    }
+    float* ring = reinterpret_cast<float*>(smem + Ly.ring + warp * p.nbs * kBoxBytes);
+    uint64_t* rfull = bars.base_full + warp * kMaxRingSlots;
+    Items L;
+    L.p = &p;
+    L.ntiles = ntiles;
+    L.last_rows = last_rows;
+    L.q = q;
+    L.h = h;
+    L.first();
+    int nl = 0, nc = 0;
+    auto issue_load = [&]() {
+      const int j = nl % p.nbs;
+      mbar_arrive_expect_tx(&rfull[j], kBoxBytes);
+      tma_load_3d(ring + j * (kBoxBytes / 4), &tm_base, lo + L.ptile() * kTileRows + kUnit * q, L.i,
+                  L.gr * p.gsize + (2 * L.k + h) * kChunk, &rfull[j], pol_first);
+      L.next();
+      ++nl;
+    };
+    if (lane == 0)
+      while (L.valid && nl < p.nbs) issue_load();
+
+    // A group's position is released (step_done) once this warp's z stores
+    // for it are complete; the wait is deferred until later stores are in
+    // flight, so the warp keeps streaming meanwhile.
+    int pending = -1, mark = 0;
+    auto release_pending = [&](int newer) {
+      if (pending < 0) return;
+      if (lane == 0) {
+        switch (min(newer, 4)) {
+          case 0: bulk_wait<0>(); break;
+          case 1: bulk_wait<1>(); break;
+          case 2: bulk_wait<2>(); break;
+          case 3: bulk_wait<3>(); break;
+          default: bulk_wait<4>(); break;
+        }
+        fence_proxy_async_all();
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.step_done[pending]);
+      pending = -1;
+    };
+
+    int slot = 0;
+    uint32_t slot_phase = 0;
+    bool ok = true;
+    for (int i = 0; ok && i < d.K; ++i) {
+      for (int gr = 0; ok && gr < p.ngroups; ++gr) {
+        const int gbase = gr * p.gsize;
+        const int nreal = group_real(p, gr);
+        double acc[kMaxGroup / kChunk];
+#pragma unroll
+        for (int k = 0; k < kMaxGroup / kChunk; ++k) acc[k] = 0.0;
+        const int nk = chunks_for(nreal, h);
+        for (int t = 0; ok && t < ntiles; ++t) {
+          const int pt = phys_tile(i, gr, p.ngroups, ntiles, t);
+          const int rows = (pt == ntiles - 1) ? last_rows : kTileRows;
+          ok = mbar_wait(&bars.acc_full[slot], slot_phase, s_abort, d.err, 0x300u);
+          if (!ok) break;
+          tc_fence_after();
+          if (kUnit * q < rows) {
+            const int v0 = lo + pt * kTileRows + kUnit * q;
+#pragma unroll
+            for (int kk = 0; kk < kMaxGroup / kChunk / 2; ++kk) {
+              if (kk < nk && ok) {
+                const int j = nc % p.nbs;
+                ok = mbar_wait(&rfull[j], (nc / p.nbs) & 1, s_abort, d.err, 0x301u);
+                if (ok) {
+                  float* box = ring + j * (kBoxBytes / 4);
+                  const int col0 = (2 * kk + h) * kChunk;
+                  uint32_t rg[32];
+                  tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(kUnit * q) << 16) +
+                                         static_cast<uint32_t>(slot * p.slot_stride + col0),
+                                     rg);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int half = 0; half < 2; ++half) {
+                    double w[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                      const int cc = half * 16 + c;
+                      const float zz = box[cc * kUnit + lane] + __uint_as_float(rg[cc]);
+                      box[cc * kUnit + lane] = zz;
+                      w[c] = (col0 + cc < nreal) ? static_cast<double>(expf(zz)) : 0.0;
+                    }
+                    acc[2 * kk + half] += reduce16(w, lane);
+                  }
+                  fence_proxy_async_shared();
+                  __syncwarp();
+                  ++nc;
+                  if (lane == 0) {
+                    tma_store_3d(&tm_z, box, v0, i, gbase + col0, pol_first);
+                    bulk_commit();
+                    bulk_wait_read<1>();
+                    while (L.valid && nl <= nc + p.nbs - 2) issue_load();
+                  }
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.acc_empty[slot]);
+          if (++slot == p.nslots) {
+            slot = 0;
+            slot_phase ^= 1u;
+          }
+          if (pending >= 0 && nc - mark > 0) release_pending(nc - mark);
+        }
+        if (!ok) break;
+        // this warp's quadrant of the slice sums of group gr
+        if ((lane & 1) == 0)
+#pragma unroll
+          for (int kk = 0; kk < kMaxGroup / kChunk / 2; ++kk)
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const int col = (2 * kk + h) * kChunk + half * 16 + (lane >> 1);
+              if (kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[2 * kk + half];
+            }
+        release_pending(0);
+        pending = gr;
+        mark = nc;
+        // with a single group the next position needs this release first
+        if (p.ngroups == 1) release_pending(0);
+      }
+    }
+    if (ok) release_pending(0);
+    if (!ok) *s_abort = 1;
+    // every copy this warp started completes before the CTA exits
+    if (lane == 0) {
+      bulk_wait<0>();
+      for (int n = nc; n < nl; ++n) mbar_drain(&rfull[n % p.nbs], (n / p.nbs) & 1, d.err, 0x302u);
+    }
+  }
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeFn>(nullptr);
+    return reinterpret_cast<EncodeFn>(f);
+  }();
+  return fn;
+}
+
+int group_size(int B) { return std::min(kMaxGroup, (B + 15) & ~15); }
+
+}  // namespace
+
+bool draft_tc_supported(const DraftArgs& a) {
+  return a.bf16 && a.r % kKStage == 0 && a.r <= 256 && a.V % kUnit == 0 && a.V >= kUnit &&
+         (a.B + group_size(a.B) - 1) / group_size(a.B) <= kMaxGroups;
+}
+
+int draft_tc_grid(int V, int sms) { return std::max(1, std::min(std::min(kMaxGrid, sms), V / kUnit)); }
+
+size_t draft_tc_extra_bytes(int B, int V, int r) {
+  (void)V;
+  const int gs = group_size(B);
+  const size_t ngroups = (B + gs - 1) / gs;
+  return align_up(ngroups * gs * r * 2, 256);
+}
+
+cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cudaStream_t stream) {
+  EncodeFn enc = encode_fn();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  TcParams p{};
+  p.d = a;
+  p.gsize = group_size(a.B);
+  p.ngroups = (a.B + p.gsize - 1) / p.gsize;
+  p.r_stages = a.r / kKStage;
+  // 32-column TMEM loads may read past a slot's N columns (masked), so slots
+  // are 32-column aligned and the last one ends inside the allocation
+  p.slot_stride = (p.gsize + 31) & ~31;
+  p.nslots = std::min(kMaxAccSlots, static_cast<int>(kTmemCols) / p.slot_stride);
+  p.image_stride = p.gsize * a.r * 2;
+  p.image = reinterpret_cast<uint8_t*>(extra);
+  p.sync_part = sync;
+  p.sync_tok = sync + a.K * p.ngroups;
+  int dev = 0, max_smem = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const int part_bytes = p.ngroups * 4 * p.gsize * 8;
+  // deepest Bf and base rings that fit, favouring at least 4 base slots
+  const int choices[][2] = {{6, 4}, {4, 4}, {6, 3}, {4, 3}, {4, 2}, {3, 2}, {2, 2}};
+  size_t smem = 0;
+  for (const auto& c : choices) {
+    const size_t need = make_layout(c[0], p.image_stride, c[1], part_bytes).total + 1024;
+    if (static_cast<int>(need) <= max_smem) {
+      p.nbf = c[0];
+      p.nbs = c[1];
+      smem = need;
+      break;
+    }
+  }
+  if (smem == 0) return cudaErrorInvalidConfiguration;
+
+  CUtensorMap tm_bf, tm_base, tm_z;
+  {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.V), static_cast<cuuint64_t>(a.r)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.V) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kKStage)};
+    cuuint32_t es[2] = {1, 1};
+    if (enc(&tm_bf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.Bf), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto enc3 = [&](CUtensorMap* tm, const float* ptr) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.V), static_cast<cuuint64_t>(a.K),
+                          static_cast<cuuint64_t>(a.B)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.V) * 4, static_cast<cuuint64_t>(a.V) * a.K * 4};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(kUnit), 1, static_cast<cuuint32_t>(kChunk)};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (!enc3(&tm_base, a.base) || !enc3(&tm_z, a.z)) return cudaErrorInvalidValue;
+
+  cudaError_t e = cudaFuncSetAttribute(draft_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, draft_tc_kernel, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (per_sm < 1 || G > per_sm * sms) return cudaErrorCooperativeLaunchTooLarge;
+  void* args[] = {&p, &tm_bf, &tm_base, &tm_z};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(draft_tc_kernel), dim3(G), dim3(kThreads), args,
+                                     smem, stream);
+}
+
+}  // namespace dspark

@@ -32,6 +32,16 @@ def test_tiny_many_seeds():
     (0, dict(B=9, K=6, V=20488, r=32, n_prof=128)),
     (1, dict(B=3, K=16, V=4104, r=256, n_prof=64)),
     (1, dict(B=130, K=2, V=8200, r=16, n_prof=512)),
+    # tensor-core draft path (bf16, r % 64 == 0, V % 32 == 0): partial last
+    # tiles, several request groups, vocabulary slices of one quadrant
+    (1, dict(B=12, K=5, V=37024, r=64, n_prof=256)),
+    (1, dict(B=130, K=3, V=8192, r=128, n_prof=600)),
+    (1, dict(B=3, K=2, V=96, r=256, n_prof=16)),
+    (1, dict(B=17, K=4, V=4096, r=192, n_prof=80)),
+    (1, dict(B=64, K=3, V=151936, r=256, n_prof=2048)),
+    # K = 32: verify lengths of 32 (33 target rows per request)
+    (1, dict(B=3, K=32, V=2048, r=64, n_prof=128)),
+    (0, dict(B=2, K=32, V=1024, r=16, n_prof=80)),
 ])
 def test_medium_ragged(like, sizes):
     t = parity.Tally()
