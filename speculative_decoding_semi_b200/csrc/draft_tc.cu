@@ -68,6 +68,7 @@ constexpr int kMaxAccSlots = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarBytes = 1024;
 
+
 struct TcParams {
   DraftArgs d;
   uint8_t* image;       // [groups][image_stride] A rows of the drawn tokens, MMA layout
@@ -193,6 +194,43 @@ struct Items {
     normalize();
   }
 };
+
+// Reduce 32 fp64 values across the 32 lanes by recursive halving: afterwards
+// lane l holds the warp-wide sum of value l.
+__device__ __forceinline__ double reduce32(double (&v)[32], int lane) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const bool up = lane & 16;
+    const double send = up ? v[j] : v[j + 16];
+    const double keep = up ? v[j + 16] : v[j];
+    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const bool up = lane & 8;
+    const double send = up ? v[j] : v[j + 8];
+    const double keep = up ? v[j + 8] : v[j];
+    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const bool up = lane & 4;
+    const double send = up ? v[j] : v[j + 4];
+    const double keep = up ? v[j + 4] : v[j];
+    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const bool up = lane & 2;
+    const double send = up ? v[j] : v[j + 2];
+    const double keep = up ? v[j + 2] : v[j];
+    v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
+  const bool up = lane & 1;
+  const double send = up ? v[0] : v[1];
+  const double keep = up ? v[1] : v[0];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+}
 
 // Reduce 16 fp64 values across the 32 lanes of a warp by recursive halving:
 // afterwards lanes 2m and 2m+1 both hold the warp-wide sum of value m.
@@ -704,6 +742,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kMaxGroup / kChunk; ++k) acc[k] = 0.0;
         const int nk = chunks_for(nreal, h);
+        // with at most one chunk per tile a lane keeps one fp64 sum per column
+        // across the tiles and the lanes are combined once, after the last
+        // tile; with two, each chunk is reduced across lanes as it is done
+        const bool per_lane = nk <= 1;
+        double cacc[kChunk];
+#pragma unroll
+        for (int c = 0; c < kChunk; ++c) cacc[c] = 0.0;
         for (int t = 0; ok && t < ntiles; ++t) {
           const int pt = phys_tile(i, gr, p.ngroups, ntiles, t);
           const int rows = (pt == ntiles - 1) ? last_rows : kTileRows;
@@ -725,17 +770,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          static_cast<uint32_t>(slot * p.slot_stride + col0),
                                      rg);
                   tmem_ld_wait();
+                  if (per_lane) {
 #pragma unroll
-                  for (int half = 0; half < 2; ++half) {
-                    double w[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                      const int cc = half * 16 + c;
-                      const float zz = box[cc * kUnit + lane] + __uint_as_float(rg[cc]);
-                      box[cc * kUnit + lane] = zz;
-                      w[c] = (col0 + cc < nreal) ? static_cast<double>(expf(zz)) : 0.0;
+                    for (int c = 0; c < kChunk; ++c) {
+                      const float zz = box[c * kUnit + lane] + __uint_as_float(rg[c]);
+                      box[c * kUnit + lane] = zz;
+                      cacc[c] += (col0 + c < nreal) ? static_cast<double>(expf(zz)) : 0.0;
                     }
-                    acc[2 * kk + half] += reduce16(w, lane);
+                  } else {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                      double w[16];
+#pragma unroll
+                      for (int c = 0; c < 16; ++c) {
+                        const int cc = half * 16 + c;
+                        const float zz = box[cc * kUnit + lane] + __uint_as_float(rg[cc]);
+                        box[cc * kUnit + lane] = zz;
+                        w[c] = (col0 + cc < nreal) ? static_cast<double>(expf(zz)) : 0.0;
+                      }
+                      acc[2 * kk + half] += reduce16(w, lane);
+                    }
                   }
                   fence_proxy_async_shared();
                   __syncwarp();
@@ -761,7 +815,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         // this warp's quadrant of the slice sums of group gr
-        if ((lane & 1) == 0)
+        if (per_lane) {
+          if (nk == 1) {
+            const double v = reduce32(cacc, lane);
+            const int col = h * kChunk + lane;
+            if (col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = v;
+          }
+        } else if ((lane & 1) == 0) {
 #pragma unroll
           for (int kk = 0; kk < kMaxGroup / kChunk / 2; ++kk)
 #pragma unroll
@@ -769,6 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int col = (2 * kk + h) * kChunk + half * 16 + (lane >> 1);
               if (kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[2 * kk + half];
             }
+        }
         release_pending(0);
         pending = gr;
         mark = nc;
