@@ -25,9 +25,11 @@ bool sizes_ok(int B, int K, int V) {
   return B >= 1 && B <= kMaxB && K >= 1 && K <= kMaxK && V >= 8 && V <= kMaxV && (V % 8) == 0;
 }
 
+// Scratch layout after kScratchOffset: schedule | verify | draft.
+size_t schedule_region(int B, int K) { return align_up(schedule_scratch_bytes(B, K), 256); }
+size_t verify_region(int B, int K, int V) { return align_up(verify_scratch_bytes(B, K, V), 256); }
 size_t scratch_bytes(int B, int K, int V, int r) {
-  return std::max({draft_scratch_bytes(B, K, V, r), verify_scratch_bytes(B, K, V),
-                   schedule_scratch_bytes(B, K)});
+  return schedule_region(B, K) + verify_region(B, K, V) + align_up(draft_scratch_bytes(B, K, V, r), 256);
 }
 
 dspark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
@@ -85,7 +87,7 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
   // tensor-core kernel; other shapes and fp32 factors the CUDA-core kernel
   const bool tc = draft_tc_supported(a);
   const int G = tc ? draft_tc_grid(V, sms) : draft_grid_size(V, sms);
-  char* scratch = ws + kScratchOffset;
+  char* scratch = ws + kScratchOffset + schedule_region(B, K) + verify_region(B, K, V);
   const size_t gmax = std::min<size_t>(kMaxGrid, V / 8);
   a.part_m = reinterpret_cast<float*>(scratch);
   a.part_S = reinterpret_cast<double*>(scratch + align_up(static_cast<size_t>(B) * gmax * sizeof(float), 256));
@@ -134,7 +136,7 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
                         u_accept, u_resample, accepted, out_tokens, n_out, workspace};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
-  if (ws_bytes < kScratchOffset + verify_scratch_bytes(B, K, V)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < kScratchOffset + schedule_region(B, K) + verify_region(B, K, V)) return DSPARK_ERR_INVALID_ARG;
   char* ws = static_cast<char*>(workspace);
   VerifyArgs a{};
   a.target = target_logits;
@@ -153,7 +155,7 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
   a.out_tokens = out_tokens;
   a.n_out = n_out;
   a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
-  return from_cuda(launch_verify(a, ws + kScratchOffset, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_verify(a, ws + kScratchOffset + schedule_region(B, K), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dspark_status dspark_l2_reserve(size_t bytes, size_t* granted) {

@@ -17,13 +17,13 @@ constexpr int kMaxV = 1 << 24;
 constexpr int kMaxR = 512;
 constexpr int kMaxScheduleItems = 16384;
 constexpr int kMaxGrid = 256;        // CTAs of the persistent draft kernel (>= SM count)
-constexpr int kVerifySeg = 4096;     // vocabulary segment of the verify kernels
 
 // -------------------------------------------------------- workspace layout
 // [0, 256)      error word: u32 code, u32 detail
 // [256, 4352)   counters of the device-wide waits (cleared by every draft launch)
-// [4352, ...)   per-call scratch (draft partials / verify partials / schedule
-//               arrays); calls on one stream reuse it in turn.
+// [4352, ...)   schedule arrays, then the verify arrays, then the draft
+//               partials (disjoint, so a round's calls never overwrite each
+//               other's data).
 constexpr size_t kErrOffset = 0;
 constexpr size_t kSyncOffset = 256;
 constexpr size_t kSyncBytes = 4096;

@@ -434,16 +434,14 @@ __device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t,
   }
 }
 
-// One warp: lane 0 waits for *ctr >= target (bounded); the result goes to all lanes.
+// One warp: every lane waits for *ctr >= target (bounded), so the warp stays
+// converged for the collective code that follows.
 __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned target, unsigned* err,
                                                   unsigned where, volatile int* abort, int lane) {
-  int ok = 1;
-  if (lane == 0) {
-    ok = wait_at_least(ctr, target, err, where) ? 1 : 0;
-    __threadfence();
-    if (!ok) *abort = 1;
-  }
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  const bool ok = __all_sync(0xffffffffu, wait_at_least(ctr, target, err, where));
+  __threadfence();
+  if (!ok && lane == 0) *abort = 1;
+  return ok;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

@@ -28,13 +28,6 @@ struct DraftArgs {
   double* part_S;   // [B][G]
 };
 
-struct VerifyDecision {
-  int acc;    // accepted drafts
-  int mode;   // 0 = residual at row acc, 1 = bonus at row acc (= L_b)
-  double M;   // max logit of the final row
-  double W;   // sum exp(x - M) of the final row
-};
-
 struct VerifyArgs {
   const float* target;
   const int64_t* row_start;
@@ -45,16 +38,11 @@ struct VerifyArgs {
   const int32_t* verify_len;
   const float* u_accept;
   const float* u_resample;
-  int B, K, V, nseg;
+  int B, K, V;
   int32_t* accepted;
   int32_t* out_tokens;
   int32_t* n_out;
   unsigned* err;
-  float* rp_m;          // [B*(K+1)][nseg]
-  double* rp_S;         // [B*(K+1)][nseg]
-  float* x_tok;         // [B*K]
-  double* seg_w;        // [B][nseg]
-  VerifyDecision* dec;  // [B]
 };
 
 struct ScheduleArgs {
@@ -76,7 +64,8 @@ size_t verify_scratch_bytes(int B, int K, int V);
 size_t schedule_scratch_bytes(int B, int K);
 
 cudaError_t launch_draft(DraftArgs a, char* scratch, cudaStream_t stream);
-cudaError_t launch_verify(VerifyArgs a, char* scratch, cudaStream_t stream);
+// `region`: the verify part of the workspace (verify_scratch_bytes bytes).
+cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream);
 cudaError_t launch_schedule(ScheduleArgs a, char* scratch, cudaStream_t stream);
 
 }  // namespace dspark

@@ -8,399 +8,860 @@
 // number; if every draft passes sample the next token from the target, else
 // resample from an adjusted distribution (here max(0, p - q) renormalised).
 //
-// Four stream-ordered kernels, one warp per unit of work:
-//   rows    : one warp per (row <= L_b, 1024-wide segment): the segment's max
-//             and fp64 sum of exp(x - max), and the logit at the drafted token.
-//             Rows are visited from the last (bonus) row down to row 0, so the
-//             rows most often rejected are the ones still in L2 afterwards.
-//   decide  : one warp per request: each row's (max, sum) from its segments,
-//             the accept decisions and the first rejection.
-//   segsum  : one warp per (request, segment): the final distribution's sum
-//             over the segment; max(0, p - q) re-reads the rejected row and its
-//             z row, the bonus reuses the row's partials.
-//   final   : one warp per request: finds the segment where u*W falls and
-//             rescans it, in coalesced rows of 128, with bit-identical weights.
+// Two launches.
+//   plan    one CTA: checks verify_len and the drafted tokens, numbers the
+//           target rows 0..L_b of every request consecutively in request
+//           order and clears the counters of the main kernel.
+//   main    one persistent cooperative CTA per SM, in five phases separated
+//           by device-wide barriers:
+//     1 rows      the target rows stream through a ring of shared-memory
+//                 stages filled by bulk asynchronous copies (one producer
+//                 warp); sixteen consumer warps, in two groups taking alternate
+//                 stages, reduce 1024-wide segments: fp64 sum of exp(x) and the
+//                 logit at the drafted token;
+//     2 row stats one warp per row: (max, sum) from the segment partials and
+//                 the accept test u * q(t) < p(t) of the row's draft;
+//     3 decide    one warp per request: the first rejection; with none, the
+//                 bonus token is drawn at once; else the request joins the
+//                 list of residual passes;
+//     4 residual  the rejected rows and their z rows stream through the same
+//                 ring: sums of max(0, p - q) over 512-wide segments;
+//     5 resample  one warp per listed request draws the resampled token.
+// The barriers fall between streaming phases, when no copy is in flight: a
+// gpu-scope fence on an SM with bulk copies in flight waits for them to land,
+// and a plain store from such an SM takes several microseconds to be seen by
+// other SMs, so cross-CTA hand-offs in the middle of a stream cost more than
+// the barriers do. Every wait is bounded and reports DSPARK_ERR_TIMEOUT.
+//
+// Weights. exp(x) is taken as 2^(x log2 e - h), one fused multiply-add and
+// one exp2f, with a base-2 shift h = 0 (a segment whose sum leaves
+// [1e-20, 1e30] is redone with its own maximum as the shift); four consecutive
+// weights are added in fp32 and the groups in fp64. The draws rescan one
+// segment with the same fp32 groups, so the segment sums and the rescans
+// agree up to the fp64 order of the groups.
+#include <algorithm>
 #include <cfloat>
+#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace dspark {
 
 namespace {
 
-constexpr int kSeg = 1024;              // segment width (32 lanes x 8 float4)
-constexpr int kVec = kSeg / 32 / 4;     // float4 per lane
-constexpr int WT = 256;                 // threads per CTA (8 warps)
+using namespace sm100;
 
-enum { kResidual = 0, kBonus = 1, kResidualAsP = 2 };
+constexpr int kSeg = 1024;                // row-pass segment: 32 lanes x 8 float4
+constexpr int kRSeg = 512;                // residual segment: 32 lanes x 4 float4
+constexpr int kCons = 8;                  // consumer warps per group (one segment each)
+constexpr int kGroups = 2;                // consumer groups, taking alternate stages
+constexpr int kProdWarp = kCons * kGroups;
+constexpr int kWarps = kProdWarp + 4;     // + producer + three more for the warp-per-unit phases
+constexpr int kThreads = kWarps * 32;
+constexpr int kRowItem = kCons * kSeg;    // logits per row item
+constexpr int kResItem = kCons * kRSeg;   // logits (and z values) per residual item
+constexpr int kStageBytes = kRowItem * 4;
+constexpr int kStages = 6;
+constexpr int kPlanThreads = 1024;
+constexpr int kRegSeg = 8;                // segment values per lane held in registers (nseg <= 256)
+constexpr int kRegWeight = 12;            // segment weights per lane held in registers
+constexpr double kSumLo = 1e-20, kSumHi = 1e30;
+constexpr float kLog2e = 1.44269504088896340736f;  // log2(e)
+constexpr double kLog2eD = 1.44269504088896340736;
 
-// Probability weights shared by `decide` and `final`, so both produce the same
-// bits: p_k = exp(x_k - m_s) * fp_s with fp_s = exp(m_s - M) / W; q_k =
-// exp(z_k - mq) * fq with mq = fp32(lse_q), fq = exp(mq - lse_q). Products and
-// differences use explicit round-to-nearest intrinsics so that no FMA
-// contraction can make the two sites differ.
-__device__ __forceinline__ double p_weight(float x, float m_s, double fp_s) {
-  return __dmul_rn(static_cast<double>(expf(x - m_s)), fp_s);
-}
-__device__ __forceinline__ double residual_weight(float x, float m_s, double fp_s, float zq, float mq,
-                                                  double fq) {
-  const double d = __dsub_rn(p_weight(x, m_s, fp_s), __dmul_rn(static_cast<double>(expf(zq - mq)), fq));
-  return d > 0.0 ? d : 0.0;
-}
+enum : int { kItemRow = 0, kItemRes = 1, kItemExit = 2 };
+enum : int { kCtlRows = 0, kCtlListed = 1, kCtlBar = 2 };  // kCtlBar..kCtlBar+3: barrier counters
 
-__device__ __forceinline__ float wmax(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ double wsum(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
+// One target row of the compact numbering.
+struct RowInfo {
+  int brl;        // b | rho << 16 | L_b << 22
+  int tok;        // drafted token tested at this row, -1 at the last row or if invalid
+  long long row;  // row index into the target logits
+};
 
-// (max, sum exp(x - max)) of a row from its segment partials, in a fixed
-// order (one warp). Up to 8 partials per lane are loaded at once.
-__device__ __forceinline__ void row_stats(const float* rp_m, const double* rp_S, int nseg, int lane, float* Mo,
-                                          double* Wo) {
-  float mv[8];
-  double sv[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int s = lane + 32 * j;
-    mv[j] = s < nseg ? __ldcg(rp_m + s) : -INFINITY;
-    sv[j] = s < nseg ? __ldcg(rp_S + s) : 0.0;
-  }
-  float m = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) m = fmaxf(m, mv[j]);
-  for (int s = lane + 256; s < nseg; s += 32) m = fmaxf(m, __ldcg(rp_m + s));
-  const float M = wmax(m);
-  double w = 0.0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (lane + 32 * j < nseg) w += __dmul_rn(sv[j], exp(static_cast<double>(mv[j]) - M));
-  for (int s = lane + 256; s < nseg; s += 32)
-    w += __dmul_rn(__ldcg(rp_S + s), exp(static_cast<double>(__ldcg(rp_m + s)) - M));
-  *Mo = M;
-  *Wo = wsum(w);
-}
+struct Desc {
+  int type, b, R, g;     // request, compact row, item index
+  int n, tok, pad0, pad1;  // logits in the item; drafted token (row items)
+  float shift[4], f[4];  // residual: per 1024-segment base-2 shift and p factor
+  float mq, fq, pad2[2];  // residual: q = 2^(z log2 e - mq) * fq
+};
 
-__global__ void __launch_bounds__(WT) verify_rows_kernel(VerifyArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * (WT / 32) + (threadIdx.x >> 5);
-  const int nw = gridDim.x * (WT / 32);
-  const long long per_rho = static_cast<long long>(a.B) * a.nseg;
-  const long long items = per_rho * (a.K + 1);
-  for (long long item = gw; item < items; item += nw) {
-    // rows from rho = K down to 0, requests and segments inside
-    const int rho = a.K - static_cast<int>(item / per_rho);
-    const long long rest = item % per_rho;
-    const int b = static_cast<int>(rest / a.nseg);
-    const int s = static_cast<int>(rest % a.nseg);
-    const int L = a.verify_len[b];
-    if (L < 0 || L > a.K) {
-      if (rho == 0 && s == 0 && lane == 0) set_error(a.err, DSPARK_ERR_DEVICE_ASSERT, 0x10000000u | b);
-      continue;
-    }
-    if (rho > L) continue;
-    const long long rowlocal = static_cast<long long>(b) * (a.K + 1) + rho;
-    const float* row = a.target + (a.row_start[b] + rho) * static_cast<long long>(a.V);
-    const int v0 = s * kSeg;
-    const int n = min(kSeg, a.V - v0);
-    float4 x[kVec];
-#pragma unroll
-    for (int k = 0; k < kVec; ++k) {
-      const int off = 4 * (k * 32 + lane);
-      x[k] = off < n ? __ldcg(reinterpret_cast<const float4*>(row + v0 + off))
-                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    }
-    float m = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < kVec; ++k) m = fmaxf(fmaxf(m, fmaxf(x[k].x, x[k].y)), fmaxf(x[k].z, x[k].w));
-    m = wmax(m);
-    double S = 0.0;
-#pragma unroll
-    for (int k = 0; k < kVec; ++k) {
-      S += static_cast<double>(expf(x[k].x - m));
-      S += static_cast<double>(expf(x[k].y - m));
-      S += static_cast<double>(expf(x[k].z - m));
-      S += static_cast<double>(expf(x[k].w - m));
-    }
-    S = wsum(S);
-    if (lane == 0) {
-      a.rp_m[rowlocal * a.nseg + s] = m;
-      a.rp_S[rowlocal * a.nseg + s] = S;
-      if (rho < L) {
-        const int t = a.tokens[b * a.K + rho];
-        if (t < 0 || t >= a.V) {
-          set_error(a.err, DSPARK_ERR_DEVICE_ASSERT, 0x20000000u | b);
-        } else if (t >= v0 && t < v0 + n) {
-          a.x_tok[b * a.K + rho] = row[t];
-        }
-      }
-    }
-  }
+struct RowStat {
+  double M, W;  // base-2 largest shift, sum of 2^(x log2 e - M)
+};
+struct ResDec {
+  int acc, R;
+  long long row;  // target row of the rejection
+  float mq, fq;
+};
+
+struct Ws {
+  RowInfo* rowinfo;  // [B*(K+1)]
+  int* rowbase;      // [B] compact index of row 0, -1 for an invalid request
+  unsigned* ctl;     // counters, cleared by the plan kernel
+  float* part_m;     // [B*(K+1)][nseg] segment base-2 shift h
+  double* part_S;    // [B*(K+1)][nseg] segment sum of 2^(x log2 e - h)
+  float* x_tok;      // [B*(K+1)] logit at the drafted token (-inf if none)
+  RowStat* rstat;    // [B*(K+1)]
+  int* accepted;     // [B*(K+1)] accept test of the row's draft
+  ResDec* dec;       // [B]
+  float2* resfac;    // [B][nseg] residual (shift, p factor) per 1024-segment
+  int* list;         // [B] requests with a residual pass
+  double* seg_w;     // [B][nrseg] residual segment sums
+};
+
+struct Params {
+  VerifyArgs a;
+  Ws w;
+  int nseg, nrseg, ngrp, nrgrp;
+};
+
+// ------------------------------------------------------------ weights
+// The fp32 weights of the target distribution p and of the residual
+// max(0, p - q); explicit rounding intrinsics keep every site bit-identical.
+__device__ __forceinline__ float p_w(float x, float h) { return exp2f(__fmaf_rn(x, kLog2e, -h)); }
+__device__ __forceinline__ float res_w(float x, float z, float h, float f, float mq, float fq) {
+  const float p = __fmul_rn(exp2f(__fmaf_rn(x, kLog2e, -h)), f);
+  const float q = __fmul_rn(exp2f(__fmaf_rn(z, kLog2e, -mq)), fq);
+  const float d = __fsub_rn(p, q);
+  return d > 0.f ? d : 0.f;
+}
+__device__ __forceinline__ float group4(float w0, float w1, float w2, float w3) {
+  return __fadd_rn(__fadd_rn(__fadd_rn(w0, w1), w2), w3);
+}
+// 2^(h - M): the scale of a segment with base-2 shift h in a row whose largest
+// shift is M (exactly 1 in the common case h == M). The rare exponential is
+// kept out of line, so the common path carries neither its instructions nor
+// their evaluation.
+__device__ __noinline__ double exp2_rare(double x) { return exp2(x); }
+__device__ __forceinline__ double seg_scale(float h, double M) {
+  if (static_cast<double>(h) == M) return 1.0;
+  return exp2_rare(static_cast<double>(h) - M);
+}
+// (shift, factor) of a 1024-segment in the residual: p = 2^(x log2 e - h) * f.
+__device__ __forceinline__ float2 res_factor(float h, double M, double W) {
+  if (h == -INFINITY) return make_float2(0.f, 0.f);
+  return make_float2(h, static_cast<float>(seg_scale(h, M) / W));
+}
+// q = exp(z - lse) = 2^(z log2 e - mq) * fq with mq = fp32(lse log2 e).
+__device__ __forceinline__ void q_factor(double lse, float* mq, float* fq) {
+  const double c = lse * kLog2eD;
+  *mq = static_cast<float>(c);
+  *fq = static_cast<float>(exp2(static_cast<double>(*mq) - c));
 }
 
-// One CTA per request: warps form the (max, sum) of rows 0..L_b in parallel,
-// then warp 0 takes the accept decisions.
-__global__ void __launch_bounds__(WT) verify_decide_kernel(VerifyArgs a) {
-  __shared__ float s_M[kMaxK + 1];
-  __shared__ double s_W[kMaxK + 1];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int b = blockIdx.x;
-  const int L = a.verify_len[b];
-  if (L < 0 || L > a.K) return;  // recorded by the rows kernel
-  for (int rho = warp; rho <= L; rho += WT / 32) {
-    const long long rl = static_cast<long long>(b) * (a.K + 1) + rho;
-    float M;
-    double W;
-    row_stats(a.rp_m + rl * a.nseg, a.rp_S + rl * a.nseg, a.nseg, lane, &M, &W);
-    if (lane == 0) {
-      s_M[rho] = M;
-      s_W[rho] = W;
-    }
+__device__ __forceinline__ float4 neg_inf4() { return make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY); }
+
+// ------------------------------------------------------------ plan kernel
+__device__ int block_exscan_int(int v, int* total, int* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
   }
   __syncthreads();
-  if (warp != 0) return;
-  bool reject = false;
-  if (lane < L) {
-    const int idx = b * a.K + lane;
-    const double p_t = exp(static_cast<double>(a.x_tok[idx]) - static_cast<double>(s_M[lane])) / s_W[lane];
-    const double uq = static_cast<double>(a.u_accept[idx]) * static_cast<double>(a.q_tok[idx]);
-    reject = !(uq < p_t);
+  if (lane == 31) red[w] = inc;
+  __syncthreads();
+  if (w == 0) {
+    const int s = lane < kPlanThreads / 32 ? red[lane] : 0;
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    if (lane < kPlanThreads / 32) red[lane] = si - s;
+    if (lane == 31) red[32] = si;
   }
-  const unsigned rej = __ballot_sync(0xffffffffu, reject);
-  const int acc = rej ? (__ffs(rej) - 1) : L;
-  const float fM = s_M[acc];
-  const double fW = s_W[acc];
-  if (lane == 0) {
-    VerifyDecision dd;
-    dd.acc = acc;
-    dd.mode = acc < L ? kResidual : kBonus;
-    dd.M = fM;
-    dd.W = fW;
-    a.dec[b] = dd;
-  }
+  __syncthreads();
+  const int ex = red[w] + inc - v;
+  *total = red[32];
+  __syncthreads();
+  return ex;
 }
 
-__global__ void __launch_bounds__(WT) verify_segsum_kernel(VerifyArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * (WT / 32) + (threadIdx.x >> 5);
-  const int nw = gridDim.x * (WT / 32);
-  const long long items = static_cast<long long>(a.B) * a.nseg;
-  for (long long item = gw; item < items; item += nw) {
-    const int b = static_cast<int>(item / a.nseg);
-    const int s = static_cast<int>(item % a.nseg);
-    const int L = a.verify_len[b];
-    if (L < 0 || L > a.K) continue;  // recorded by the rows kernel
-    const VerifyDecision dd = a.dec[b];
-    const int acc = dd.acc, mode = dd.mode;
-    const long long rl = static_cast<long long>(b) * (a.K + 1) + acc;
-    const float M = dd.M;
-    const double W = dd.W;
-    const float m_s = __ldcg(a.rp_m + rl * a.nseg + s);
-    const double fp_s = exp(static_cast<double>(m_s) - M) / W;
-    if (mode == kBonus) {
-      if (lane == 0) a.seg_w[static_cast<long long>(b) * a.nseg + s] = __dmul_rn(__ldcg(a.rp_S + rl * a.nseg + s), fp_s);
-      continue;
+__global__ void __launch_bounds__(kPlanThreads) verify_plan_kernel(Params p) {
+  __shared__ int red[33];
+  // the main kernel may start its prologue now; it waits for this grid's
+  // results before reading them
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const VerifyArgs& a = p.a;
+  int carry = 0;
+  for (int base = 0; base < a.B; base += kPlanThreads) {
+    const int b = base + threadIdx.x;
+    int L = -1;
+    bool valid = false;
+    if (b < a.B) {
+      L = a.verify_len[b];
+      valid = L >= 0 && L <= a.K;
+      if (!valid) set_error(a.err, DSPARK_ERR_DEVICE_ASSERT, 0x10000000u | static_cast<unsigned>(b));
     }
-    const float* row = a.target + (a.row_start[b] + acc) * static_cast<long long>(a.V);
-    const float* zrow = a.z + (static_cast<long long>(b) * a.K + acc) * a.V;
-    const double lq = a.lse_q[b * a.K + acc];
-    const float mq = static_cast<float>(lq);
-    const double fq = exp(static_cast<double>(mq) - lq);
-    const int v0 = s * kSeg;
-    const int n = min(kSeg, a.V - v0);
-    float4 x[kVec], zz[kVec];
-#pragma unroll
-    for (int k = 0; k < kVec; ++k) {
-      const int off = 4 * (k * 32 + lane);
-      if (off < n) {
-        x[k] = __ldcg(reinterpret_cast<const float4*>(row + v0 + off));
-        zz[k] = __ldcs(reinterpret_cast<const float4*>(zrow + v0 + off));
+    int total;
+    const int ex = block_exscan_int(valid ? L + 1 : 0, &total, red);
+    if (b < a.B) {
+      const int r0 = carry + ex;
+      p.w.rowbase[b] = valid ? r0 : -1;
+      if (valid) {
+        for (int rho = 0; rho <= L; ++rho) {
+          int tok = -1;
+          if (rho < L) {
+            tok = a.tokens[static_cast<long long>(b) * a.K + rho];
+            if (tok < 0 || tok >= a.V) {
+              set_error(a.err, DSPARK_ERR_DEVICE_ASSERT, 0x20000000u | static_cast<unsigned>(b));
+              tok = -1;  // x_tok stays -inf: p(t) = 0 and the draft is rejected
+            }
+          }
+          RowInfo ri;
+          ri.brl = b | (rho << 16) | (L << 22);
+          ri.tok = tok;
+          ri.row = a.row_start[b] + rho;
+          p.w.rowinfo[r0 + rho] = ri;
+          p.w.x_tok[r0 + rho] = -INFINITY;
+        }
       }
     }
-    double w = 0.0;
-#pragma unroll
-    for (int k = 0; k < kVec; ++k) {
-      const int off = 4 * (k * 32 + lane);
-      if (off < n) {
-        w += residual_weight(x[k].x, m_s, fp_s, zz[k].x, mq, fq);
-        w += residual_weight(x[k].y, m_s, fp_s, zz[k].y, mq, fq);
-        w += residual_weight(x[k].z, m_s, fp_s, zz[k].z, mq, fq);
-        w += residual_weight(x[k].w, m_s, fp_s, zz[k].w, mq, fq);
-      }
-    }
-    w = wsum(w);
-    if (lane == 0) a.seg_w[static_cast<long long>(b) * a.nseg + s] = w;
+    carry += total;
   }
+  if (threadIdx.x < 8) p.w.ctl[threadIdx.x] = threadIdx.x == kCtlRows ? static_cast<unsigned>(carry) : 0u;
 }
 
-__global__ void __launch_bounds__(WT) verify_final_kernel(VerifyArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int b = blockIdx.x * (WT / 32) + (threadIdx.x >> 5);
-  if (b >= a.B) return;
-  const int L = a.verify_len[b];
-  if (L < 0 || L > a.K) return;
-  const VerifyDecision d = a.dec[b];
-  const int acc = d.acc;
-  int mode = d.mode;
-  const long long rl = static_cast<long long>(b) * (a.K + 1) + acc;
-  const float* row = a.target + (a.row_start[b] + acc) * static_cast<long long>(a.V);
-  const float* zrow = a.z + (static_cast<long long>(b) * a.K + min(acc, a.K - 1)) * a.V;
-  const double lq = a.lse_q[b * a.K + min(acc, a.K - 1)];
-  const float mq = static_cast<float>(lq);
-  const double fq = exp(static_cast<double>(mq) - lq);
-  const int nseg = a.nseg;
-  // segment totals of the final distribution in segment order, lane-blocked
+// ------------------------------------------------------ warp-level helpers
+// Inverse CDF over nseg segment weights (one warp; `weight(q)` must return the
+// same value whenever called): the first segment whose inclusive running sum
+// exceeds u * total with a positive weight, else (rounding) the last positive
+// one. Lane l owns a contiguous block of segments. *rem = u * total minus the
+// weight before the chosen segment. Returns -1 if total <= 0.
+template <class Weight>
+__device__ int pick_segment(int nseg, float u, int lane, Weight weight, double* rem) {
   const int per = (nseg + 31) / 32;
-  const int s_lo = min(nseg, lane * per), s_hi = min(nseg, s_lo + per);
-  auto seg_total = [&](int q) -> double {
-    if (mode == kResidual) return __ldcg(a.seg_w + static_cast<long long>(b) * nseg + q);
-    const double fp = exp(static_cast<double>(__ldcg(a.rp_m + rl * nseg + q)) - d.M) / d.W;
-    return __dmul_rn(__ldcg(a.rp_S + rl * nseg + q), fp);
-  };
+  const int lo = min(nseg, lane * per), hi = min(nseg, lo + per);
+  const bool cached = per <= kRegWeight;
+  double wv[kRegWeight];
   double local = 0.0;
-  for (int q = s_lo; q < s_hi; ++q) local += seg_total(q);
-  double run = 0.0, ex = 0.0;
-  for (int l = 0; l < 32; ++l) {
-    const double v = __shfl_sync(0xffffffffu, local, l);
-    if (l == lane) ex = run;
-    run += v;
-  }
-  if (mode == kResidual && !(run > 0.0)) {
-    // max(0, p - q) vanished (only possible through rounding): sample p
-    mode = kResidualAsP;
-    local = 0.0;
-    for (int q = s_lo; q < s_hi; ++q) local += seg_total(q);
-    run = 0.0;
-    for (int l = 0; l < 32; ++l) {
-      const double v = __shfl_sync(0xffffffffu, local, l);
-      if (l == lane) ex = run;
-      run += v;
+  if (cached) {
+    // unconditional calls on clamped indices, so that every load issues at once
+#pragma unroll
+    for (int i = 0; i < kRegWeight; ++i) wv[i] = weight(min(lo + i, nseg - 1));
+#pragma unroll
+    for (int i = 0; i < kRegWeight; ++i) {
+      if (lo + i >= hi) wv[i] = 0.0;
+      local += wv[i];
     }
+  } else {
+    for (int q = lo; q < hi; ++q) local += weight(q);
   }
-  const double thr = static_cast<double>(a.u_resample[b]) * run;
-  // first segment whose inclusive prefix exceeds thr
-  int cand = 0x7fffffff;
-  double cand_ex = 0.0;
-  {
-    double c = ex;
-    for (int q = s_lo; q < s_hi; ++q) {
-      const double v = seg_total(q);
-      if (c + v > thr && v > 0.0) {
+  const double inc = warp_inclusive_scan(local);
+  double ex = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) ex = 0.0;
+  const double total = __shfl_sync(0xffffffffu, inc, 31);
+  if (!(total > 0.0)) return -1;
+  const double thr = static_cast<double>(u) * total;
+  int cand = INT_MAX, lastq = -1;
+  double cand_ex = 0.0, last_ex = 0.0, c = ex;
+  auto visit = [&](int q, double v) {
+    if (v > 0.0) {
+      if (cand == INT_MAX && c + v > thr) {
         cand = q;
         cand_ex = c;
-        break;
       }
-      c += v;
+      lastq = q;
+      last_ex = c;
     }
-  }
-  int seg = cand;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) seg = min(seg, __shfl_xor_sync(0xffffffffu, seg, o));
-  double seg_ex;
-  if (seg == 0x7fffffff) {
-    // rounding: the last segment, with its exclusive prefix
-    seg = nseg - 1;
-    double e = 0.0;
-    if (seg >= s_lo && seg < s_hi) {
-      e = ex;
-      for (int q = s_lo; q < seg; ++q) e += seg_total(q);
-    }
-    const int owner = min(31, seg / max(per, 1));
-    seg_ex = __shfl_sync(0xffffffffu, e, owner);
-  } else {
-    const int owner = min(31, seg / max(per, 1));
-    seg_ex = __shfl_sync(0xffffffffu, cand_ex, owner);
-  }
-  const double R = thr - seg_ex;
-  // rescan the segment in rows of 128 (lane l: elements 4l..4l+3 of a row),
-  // with the weights of the segsum kernel, in vocabulary order
-  const int v0 = seg * kSeg;
-  const int n = min(kSeg, a.V - v0);
-  const float m_s = __ldcg(a.rp_m + rl * nseg + seg);
-  const double fp_s = exp(static_cast<double>(m_s) - d.M) / d.W;
-  struct XZ {
-    float4 x, z;
+    c += v;
   };
+  if (cached) {
+#pragma unroll
+    for (int i = 0; i < kRegWeight; ++i)
+      if (lo + i < hi) visit(lo + i, wv[i]);
+  } else {
+    for (int q = lo; q < hi; ++q) visit(q, weight(q));
+  }
+  int seg = warp_min_int(cand);
+  double seg_ex;
+  if (seg != INT_MAX) {
+    seg_ex = __shfl_sync(0xffffffffu, cand_ex, seg / per);
+  } else {
+    seg = warp_max_int(lastq);
+    if (seg < 0) return -1;
+    seg_ex = __shfl_sync(0xffffffffu, last_ex, seg / per);
+  }
+  *rem = thr - seg_ex;
+  return seg;
+}
+
+// First element of a run of n <= 32 * E elements whose running sum of
+// weights exceeds R with a positive weight, or -1 (then *last = the last
+// positive one); one warp. Lane l owns elements [E l, E l + E): w[] holds
+// their fp32 weights (zero past n). Four consecutive weights form one fp32
+// group exactly as in the segment sums; the groups accumulate in fp64, one
+// warp-wide scan over the lanes' totals, then a search inside one lane.
+template <int E>
+__device__ int rescan(int n, int lane, double R, const float (&w)[E], int* last) {
+  float c[E];  // inclusive fp32 sums within each group of four
+  double lsum = 0.0;
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    c[4 * k] = w[4 * k];
+    c[4 * k + 1] = __fadd_rn(c[4 * k], w[4 * k + 1]);
+    c[4 * k + 2] = __fadd_rn(c[4 * k + 1], w[4 * k + 2]);
+    c[4 * k + 3] = __fadd_rn(c[4 * k + 2], w[4 * k + 3]);
+    lsum += static_cast<double>(c[4 * k + 3]);
+  }
+  const double inc = warp_inclusive_scan(lsum);
+  double before = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) before = 0.0;
+  int hit = -1, lp = -1;
+  if (before + lsum > R) {
+#pragma unroll
+    for (int k = 0; k < E / 4; ++k) {
+      if (hit < 0) {
+#pragma unroll
+        for (int j = 3; j >= 0; --j)
+          if (w[4 * k + j] > 0.f && before + static_cast<double>(c[4 * k + j]) > R) hit = 4 * k + j;
+        before += static_cast<double>(c[4 * k + 3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (w[e] > 0.f) lp = E * lane + e;
+  *last = warp_max_int(lp);
+  const unsigned hits = __ballot_sync(0xffffffffu, hit >= 0);
+  if (!hits) return -1;
+  const int hl = __ffs(hits) - 1;
+  return E * hl + __shfl_sync(0xffffffffu, hit, hl);
+}
+
+// Phase 2, one warp: (M, W) of compact row R from its segment partials, and
+// the accept test of the row's draft.
+__device__ void row_stats(const Params& P, int R, int lane) {
+  const VerifyArgs& a = P.a;
+  const RowInfo ri = P.w.rowinfo[R];
+  const int b = ri.brl & 0xffff, rho = (ri.brl >> 16) & 63, L = ri.brl >> 22;
+  const float* pm = P.w.part_m + static_cast<long long>(R) * P.nseg;
+  const double* pS = P.w.part_S + static_cast<long long>(R) * P.nseg;
+  float m = -INFINITY;
+  double w = 0.0;
+  if (P.nseg <= 32 * kRegSeg) {
+    float mv[kRegSeg];
+    double sv[kRegSeg];
+#pragma unroll
+    for (int j = 0; j < kRegSeg; ++j) {
+      const int s = lane + 32 * j;
+      mv[j] = s < P.nseg ? __ldcg(pm + s) : -INFINITY;
+      sv[j] = s < P.nseg ? __ldcg(pS + s) : 0.0;
+    }
+#pragma unroll
+    for (int j = 0; j < kRegSeg; ++j) m = fmaxf(m, mv[j]);
+    m = warp_max(m);
+#pragma unroll
+    for (int j = 0; j < kRegSeg; ++j)
+      if (sv[j] > 0.0) w += __dmul_rn(sv[j], seg_scale(mv[j], m));
+  } else {
+    for (int s = lane; s < P.nseg; s += 32) m = fmaxf(m, __ldcg(pm + s));
+    m = warp_max(m);
+    for (int s = lane; s < P.nseg; s += 32) {
+      const double S = __ldcg(pS + s);
+      if (S > 0.0) w += __dmul_rn(S, seg_scale(__ldcg(pm + s), m));
+    }
+  }
+  const double W = warp_sum(w);
+  if (lane == 0) {
+    RowStat st;
+    st.M = m;
+    st.W = W;
+    P.w.rstat[R] = st;
+    int accept = 1;
+    if (rho < L) {
+      const long long idx = static_cast<long long>(b) * a.K + rho;
+      const double p_t = exp2(static_cast<double>(__ldcg(P.w.x_tok + R)) * kLog2eD - static_cast<double>(m)) / W;
+      const double uq = static_cast<double>(a.u_accept[idx]) * static_cast<double>(a.q_tok[idx]);
+      accept = uq < p_t ? 1 : 0;
+    }
+    P.w.accepted[R] = accept;
+  }
+}
+
+// Draw from p of compact row R (the bonus row, or a rejected row whose
+// residual vanished) with the row pass's segment sums; one warp.
+__device__ __noinline__ int sample_p(const Params& P, int R, float u, int lane) {
+  const VerifyArgs& a = P.a;
+  const float* pm = P.w.part_m + static_cast<long long>(R) * P.nseg;
+  const double* pS = P.w.part_S + static_cast<long long>(R) * P.nseg;
+  const double M = __ldcg(&P.w.rstat[R].M), W = __ldcg(&P.w.rstat[R].W);
+  const long long row = P.w.rowinfo[R].row;
+  auto weight = [&](int q) -> double {
+    const double S = __ldcg(pS + q);
+    const float h = __ldcg(pm + q);
+    return S > 0.0 ? __dmul_rn(S, seg_scale(h, M) / W) : 0.0;
+  };
+  double rem = 0.0;
+  const int seg = pick_segment(P.nseg, u, lane, weight, &rem);
+  if (seg < 0) return 0;  // no positive weight: degenerate row
+  const float m_s = __ldcg(pm + seg);
+  const double Rs = rem / (seg_scale(m_s, M) / W);
+  const float* x = a.target + row * a.V + static_cast<long long>(seg) * kSeg;
+  const int n = min(kSeg, a.V - seg * kSeg);
+  constexpr int E = kSeg / 32;
+  float w[E];
+#pragma unroll
+  for (int k = 0; k < E / 4; ++k) {
+    const int e = E * lane + 4 * k;
+    const float4 v = e < n ? __ldcg(reinterpret_cast<const float4*>(x + e)) : neg_inf4();
+    w[4 * k] = p_w(v.x, m_s);
+    w[4 * k + 1] = p_w(v.y, m_s);
+    w[4 * k + 2] = p_w(v.z, m_s);
+    w[4 * k + 3] = p_w(v.w, m_s);
+  }
   int last = -1;
-  int k = scan_rows128<kSeg / 128, XZ>(
-      n, lane, R,
-      [&](int e) {
-        XZ v;
-        v.x = __ldcg(reinterpret_cast<const float4*>(row + v0 + e));
-        v.z = mode == kResidual ? __ldcg(reinterpret_cast<const float4*>(zrow + v0 + e)) : v.x;
-        return v;
-      },
-      [&](const XZ& v, double(&w)[4]) {
-        if (mode == kResidual) {
-          w[0] = residual_weight(v.x.x, m_s, fp_s, v.z.x, mq, fq);
-          w[1] = residual_weight(v.x.y, m_s, fp_s, v.z.y, mq, fq);
-          w[2] = residual_weight(v.x.z, m_s, fp_s, v.z.z, mq, fq);
-          w[3] = residual_weight(v.x.w, m_s, fp_s, v.z.w, mq, fq);
-        } else {
-          w[0] = p_weight(v.x.x, m_s, fp_s);
-          w[1] = p_weight(v.x.y, m_s, fp_s);
-          w[2] = p_weight(v.x.z, m_s, fp_s);
-          w[3] = p_weight(v.x.w, m_s, fp_s);
-        }
-      },
-      &last);
-  if (k < 0) k = max(last, 0);  // rounding: the last positive weight
+  int k = rescan<E>(n, lane, Rs, w, &last);
+  if (k < 0) k = max(last, 0);
+  return seg * kSeg + k;
+}
+
+// Emits request b's accepted drafts and the drawn token.
+__device__ void write_output(const Params& P, int b, int acc, int tok, int lane) {
+  const VerifyArgs& a = P.a;
   int32_t* out = a.out_tokens + static_cast<long long>(b) * (a.K + 1);
-  for (int j = lane; j <= a.K; j += 32) out[j] = j < acc ? a.tokens[b * a.K + j] : (j == acc ? v0 + k : -1);
+  // j = 32 (K = 32 only) is never an accepted draft, since acc <= K
+  for (int j = lane; j <= a.K; j += 32)
+    out[j] = j < acc ? a.tokens[static_cast<long long>(b) * a.K + j] : (j == acc ? tok : -1);
   if (lane == 0) {
     a.accepted[b] = acc;
     a.n_out[b] = acc + 1;
   }
 }
 
-}  // namespace
-
-size_t verify_scratch_bytes(int B, int K, int V) {
-  const size_t nseg = (V + kSeg - 1) / kSeg;
-  const size_t rows = static_cast<size_t>(B) * (K + 1);
-  size_t off = 0;
-  off = align_up(off + rows * nseg * sizeof(float), 256);
-  off = align_up(off + rows * nseg * sizeof(double), 256);
-  off = align_up(off + static_cast<size_t>(B) * K * sizeof(float), 256);
-  off = align_up(off + static_cast<size_t>(B) * nseg * sizeof(double), 256);
-  off = align_up(off + static_cast<size_t>(B) * sizeof(VerifyDecision), 256);
-  return off;
+// Phase 3, one warp: request b's first rejection; the bonus draw, or the
+// residual pass's inputs and a place in the list.
+__device__ __noinline__ void decide(const Params& P, int b, int lane) {
+  const VerifyArgs& a = P.a;
+  const int r0 = P.w.rowbase[b];
+  if (r0 < 0) return;  // invalid request (recorded by the plan kernel)
+  const int L = a.verify_len[b];
+  // drafted rows are rho < L <= 32: one lane each
+  const bool rej = lane < L && __ldcg(P.w.accepted + r0 + lane) == 0;
+  const unsigned m = __ballot_sync(0xffffffffu, rej);
+  const int acc = m ? __ffs(m) - 1 : L;
+  const int R = r0 + acc;
+  if (acc == L) {
+    const int tok = sample_p(P, R, a.u_resample[b], lane);
+    write_output(P, b, L, tok, lane);
+    return;
+  }
+  const double M = __ldcg(&P.w.rstat[R].M), W = __ldcg(&P.w.rstat[R].W);
+  const float* pm = P.w.part_m + static_cast<long long>(R) * P.nseg;
+  float2* rf = P.w.resfac + static_cast<long long>(b) * P.nseg;
+  for (int q0 = 0; q0 < P.nseg; q0 += 32 * kRegSeg) {
+    float mv[kRegSeg];
+#pragma unroll
+    for (int j = 0; j < kRegSeg; ++j) {
+      const int q = q0 + lane + 32 * j;
+      mv[j] = q < P.nseg ? __ldcg(pm + q) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kRegSeg; ++j) {
+      const int q = q0 + lane + 32 * j;
+      if (q < P.nseg) rf[q] = res_factor(mv[j], M, W);
+    }
+  }
+  if (lane == 0) {
+    ResDec d;
+    d.acc = acc;
+    d.R = R;
+    d.row = P.w.rowinfo[R].row;
+    q_factor(a.lse_q[static_cast<long long>(b) * a.K + acc], &d.mq, &d.fq);
+    P.w.dec[b] = d;
+    P.w.list[atomicAdd(P.w.ctl + kCtlListed, 1u)] = b;
+  }
 }
 
-cudaError_t launch_verify(VerifyArgs a, char* scratch, cudaStream_t stream) {
-  a.nseg = (a.V + kSeg - 1) / kSeg;
-  const size_t nseg = a.nseg;
-  const size_t rows = static_cast<size_t>(a.B) * (a.K + 1);
+// Phase 5, one warp: the resampled token of listed request b.
+__device__ __noinline__ void resample(const Params& P, int b, int lane) {
+  const VerifyArgs& a = P.a;
+  const ResDec d = P.w.dec[b];
+  const double* sw = P.w.seg_w + static_cast<long long>(b) * P.nrseg;
+  const float u = a.u_resample[b];
+  double rem = 0.0;
+  const int seg = pick_segment(P.nrseg, u, lane, [&](int q) -> double { return __ldcg(sw + q); }, &rem);
+  int tok;
+  if (seg < 0) {
+    tok = sample_p(P, d.R, u, lane);  // the residual vanished (rounding): draw from p
+  } else {
+    const float2 sf = __ldcg(P.w.resfac + static_cast<long long>(b) * P.nseg + seg / 2);
+    const long long v0 = static_cast<long long>(seg) * kRSeg;
+    const float* x = a.target + d.row * a.V + v0;
+    const float* zr = a.z + (static_cast<long long>(b) * a.K + d.acc) * a.V + v0;
+    const int n = min(kRSeg, a.V - static_cast<int>(v0));
+    constexpr int E = kRSeg / 32;
+    float w[E];
+#pragma unroll
+    for (int k = 0; k < E / 4; ++k) {
+      const int e = E * lane + 4 * k;
+      const float4 xv = e < n ? __ldcg(reinterpret_cast<const float4*>(x + e)) : neg_inf4();
+      const float4 zv = e < n ? __ldcg(reinterpret_cast<const float4*>(zr + e)) : neg_inf4();
+      w[4 * k] = res_w(xv.x, zv.x, sf.x, sf.y, d.mq, d.fq);
+      w[4 * k + 1] = res_w(xv.y, zv.y, sf.x, sf.y, d.mq, d.fq);
+      w[4 * k + 2] = res_w(xv.z, zv.z, sf.x, sf.y, d.mq, d.fq);
+      w[4 * k + 3] = res_w(xv.w, zv.w, sf.x, sf.y, d.mq, d.fq);
+    }
+    int last = -1;
+    int k = rescan<E>(n, lane, rem, w, &last);
+    if (k < 0) k = max(last, 0);
+    tok = static_cast<int>(v0) + k;
+  }
+  write_output(P, b, d.acc, tok, lane);
+}
+
+// -------------------------------------------------------- consumer bodies
+// Segment w of a row item: sum of exp(x - shift) and the drafted token's logit.
+__device__ void consume_row(const Params& P, const Desc& ds, const float* stage, uint64_t* empty, int w, int lane) {
+  const int off_w = w * kSeg;
+  const int nw = min(kSeg, ds.n - off_w);  // <= 0 past the end of the row
+  const float* sp = stage + off_w;
+  float4 x[kSeg / 128];
+#pragma unroll
+  for (int k = 0; k < kSeg / 128; ++k) {
+    const int e = k * 128 + 4 * lane;
+    x[k] = e < nw ? reinterpret_cast<const float4*>(sp)[k * 32 + lane] : neg_inf4();
+  }
+  const int v_w = ds.g * kRowItem + off_w;
+  const bool has_tok = nw > 0 && ds.tok >= v_w && ds.tok < v_w + nw;
+  float xt = 0.f;
+  if (has_tok && lane == 0) xt = sp[ds.tok - v_w];
+  const int R = ds.R, g = ds.g;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty);
+  if (nw <= 0) return;
+  double S = 0.0;
+#pragma unroll
+  for (int k = 0; k < kSeg / 128; ++k)
+    S += static_cast<double>(group4(p_w(x[k].x, 0.f), p_w(x[k].y, 0.f), p_w(x[k].z, 0.f), p_w(x[k].w, 0.f)));
+  S = warp_sum(S);
+  float m = 0.f;
+  if (!(S >= kSumLo && S <= kSumHi)) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kSeg / 128; ++k) mx = fmaxf(fmaxf(mx, fmaxf(x[k].x, x[k].y)), fmaxf(x[k].z, x[k].w));
+    mx = warp_max(mx);
+    S = 0.0;
+    m = -INFINITY;
+    if (mx != -INFINITY) {
+      m = __fmul_rn(mx, kLog2e);
+#pragma unroll
+      for (int k = 0; k < kSeg / 128; ++k)
+        S += static_cast<double>(group4(p_w(x[k].x, m), p_w(x[k].y, m), p_w(x[k].z, m), p_w(x[k].w, m)));
+      S = warp_sum(S);
+    }
+  }
+  if (lane == 0) {
+    const long long idx = static_cast<long long>(R) * P.nseg + g * kCons + w;
+    P.w.part_m[idx] = m;
+    P.w.part_S[idx] = S;
+    if (has_tok) P.w.x_tok[R] = xt;
+  }
+}
+
+// Segment w of a residual item: sum of max(0, p - q).
+__device__ void consume_res(const Params& P, const Desc& ds, const float* stage, uint64_t* empty, int w, int lane) {
+  const int off_w = w * kRSeg;
+  const int nw = min(kRSeg, ds.n - off_w);
+  const float* sp = stage + off_w;
+  const float* sz = stage + kResItem + off_w;
+  float4 x[kRSeg / 128], z[kRSeg / 128];
+#pragma unroll
+  for (int k = 0; k < kRSeg / 128; ++k) {
+    const int e = k * 128 + 4 * lane;
+    x[k] = e < nw ? reinterpret_cast<const float4*>(sp)[k * 32 + lane] : neg_inf4();
+    z[k] = e < nw ? reinterpret_cast<const float4*>(sz)[k * 32 + lane] : neg_inf4();
+  }
+  const float sh = ds.shift[w / 2], f = ds.f[w / 2], mq = ds.mq, fq = ds.fq;
+  const int b = ds.b, g = ds.g;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty);
+  if (nw <= 0) return;
+  double S = 0.0;
+#pragma unroll
+  for (int k = 0; k < kRSeg / 128; ++k)
+    S += static_cast<double>(group4(res_w(x[k].x, z[k].x, sh, f, mq, fq), res_w(x[k].y, z[k].y, sh, f, mq, fq),
+                                    res_w(x[k].z, z[k].z, sh, f, mq, fq), res_w(x[k].w, z[k].w, sh, f, mq, fq)));
+  S = warp_sum(S);
+  if (lane == 0) P.w.seg_w[static_cast<long long>(b) * P.nrseg + g * kCons + w] = S;
+}
+
+// ------------------------------------------------------------ main kernel
+struct Smem {
+  uint64_t full[kStages], empty[kStages];
+  Desc desc[kStages];
+  int abort;
+};
+
+// Device-wide barrier k (bounded): every thread's earlier writes are visible
+// to every thread after it. Called between streaming phases, with no copy in
+// flight.
+__device__ bool grid_barrier(const Params& P, int k, int* s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    red_release_gpu_add(P.w.ctl + kCtlBar + k, 1u);
+    const bool ok = wait_at_least(P.w.ctl + kCtlBar + k, gridDim.x, P.a.err, 0x500u + k);
+    __threadfence();
+    *s_flag = ok ? 1 : 0;
+  }
+  __syncthreads();
+  return *s_flag != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_constant__ Params P) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  float* stages = reinterpret_cast<float*>(smem);
+  Smem& S = *reinterpret_cast<Smem*>(smem + kStages * kStageBytes);
+  __shared__ int s_flag;
+  const VerifyArgs& a = P.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  // warp-per-unit phases: unit u goes to CTA u % G, warp u / G, so that
+  // consecutive units (rows, requests) land on different SMs
+  const int gw = warp * G + c, NW = G * kWarps;
+  volatile int* abort = &S.abort;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], kCons);
+    }
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  // the plan kernel's results (programmatic dependent launch; a no-op when
+  // launched without it)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();
+  const int n_rows = static_cast<int>(P.w.ctl[kCtlRows]);
+  // producer: items issued; consumer group g: index of its next item
+  uint32_t seq = warp < kProdWarp ? static_cast<uint32_t>(warp / kCons) : 0u;
+
+  // One streaming phase: the producer issues this CTA's items (fill(item,
+  // desc, dst, full) fills the descriptor and starts the copies), then one
+  // exit marker per consumer group; consumers reduce the items.
+  auto stream = [&](long long n_items, auto fill, auto consume) -> bool {
+    if (warp == kProdWarp) {
+      bool ok = true;
+      auto claim = [&](int* s) -> bool {
+        *s = seq % kStages;
+        return __all_sync(0xffffffffu, mbar_wait(&S.empty[*s], ((seq / kStages) & 1u) ^ 1u, abort, a.err, 0x402u));
+      };
+      for (long long item = c; ok && item < n_items; item += G) {
+        int s;
+        ok = claim(&s);
+        if (!ok) break;
+        if (lane == 0) fill(item, S.desc[s], stages + static_cast<size_t>(s) * kRowItem, &S.full[s]);
+        ++seq;
+      }
+      for (int k = 0; ok && k < kGroups; ++k) {
+        int s;
+        ok = claim(&s);
+        if (!ok) break;
+        if (lane == 0) {
+          S.desc[s].type = kItemExit;
+          mbar_arrive(&S.full[s]);
+        }
+        ++seq;
+      }
+      if (!ok && lane == 0) *abort = 1;
+      return ok;
+    }
+    if (warp < kProdWarp) {
+      const int w = warp % kCons;
+      for (;; seq += kGroups) {
+        const int s = seq % kStages;
+        // every lane waits: a warp left waiting on one lane runs its next
+        // collective code diverged and several times slower
+        if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], (seq / kStages) & 1u, abort, a.err, 0x400u))) return false;
+        const Desc& ds = S.desc[s];
+        if (ds.type == kItemExit) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.empty[s]);
+          seq += kGroups;
+          return true;
+        }
+        consume(ds, stages + static_cast<size_t>(s) * kRowItem, &S.empty[s], w);
+      }
+    }
+    return true;
+  };
+
+  // ---- phase 1: target rows
+  const long long n_row_items = static_cast<long long>(n_rows) * P.ngrp;
+  bool ok = stream(
+      n_row_items,
+      [&](long long item, Desc& ds, float* dst, uint64_t* full) {
+        const int R = static_cast<int>(item / P.ngrp), g = static_cast<int>(item % P.ngrp);
+        const RowInfo ri = P.w.rowinfo[R];
+        const int v0 = g * kRowItem, n = min(kRowItem, a.V - v0);
+        ds.type = kItemRow;
+        ds.b = ri.brl & 0xffff;
+        ds.R = R;
+        ds.g = g;
+        ds.n = n;
+        ds.tok = ri.tok;
+        const uint32_t bytes = static_cast<uint32_t>(n) * 4u;
+        mbar_arrive_expect_tx(full, bytes);
+        bulk_load(dst, a.target + ri.row * a.V + v0, bytes, full);
+      },
+      [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_row(P, ds, stage, empty, w, lane); });
+  ok = __syncthreads_and(ok) && grid_barrier(P, 0, &s_flag);
+
+  // ---- phase 2: row statistics and accept tests
+  if (ok)
+    for (int R = gw; R < n_rows; R += NW) row_stats(P, R, lane);
+  ok = ok && grid_barrier(P, 1, &s_flag);
+
+  // ---- phase 3: decisions, bonus draws, residual list
+  if (ok)
+    for (int b = gw; b < a.B; b += NW) decide(P, b, lane);
+  ok = ok && grid_barrier(P, 2, &s_flag);
+
+  // ---- phase 4: residual segment sums of the listed requests
+  const int n_listed = ok ? static_cast<int>(__ldcg(P.w.ctl + kCtlListed)) : 0;
+  if (ok) {
+    const uint64_t pol_first = policy_evict_first();
+    ok = stream(
+        static_cast<long long>(n_listed) * P.nrgrp,
+        [&](long long item, Desc& ds, float* dst, uint64_t* full) {
+          const int e = static_cast<int>(item / P.nrgrp), g = static_cast<int>(item % P.nrgrp);
+          const int b = __ldcg(P.w.list + e);
+          const ResDec d = P.w.dec[b];
+          const int v0 = g * kResItem, n = min(kResItem, a.V - v0);
+          ds.type = kItemRes;
+          ds.b = b;
+          ds.R = d.R;
+          ds.g = g;
+          ds.n = n;
+          ds.tok = -1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int q = g * 4 + i;
+            const float2 f =
+                q < P.nseg ? __ldcg(P.w.resfac + static_cast<long long>(b) * P.nseg + q) : make_float2(0.f, 0.f);
+            ds.shift[i] = f.x;
+            ds.f[i] = f.y;
+          }
+          ds.mq = d.mq;
+          ds.fq = d.fq;
+          const uint32_t bytes = static_cast<uint32_t>(n) * 4u;
+          mbar_arrive_expect_tx(full, 2u * bytes);
+          bulk_load(dst, a.target + d.row * a.V + v0, bytes, full);
+          bulk_load_hint(dst + kResItem, a.z + (static_cast<long long>(b) * a.K + d.acc) * a.V + v0, bytes, full,
+                         pol_first);
+        },
+        [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_res(P, ds, stage, empty, w, lane); });
+    ok = __syncthreads_and(ok) && grid_barrier(P, 3, &s_flag);
+  }
+
+  // ---- phase 5: resampled tokens
+  if (ok)
+    for (int e = gw; e < n_listed; e += NW) resample(P, __ldcg(P.w.list + e), lane);
+
+  // copies still in flight (after an abort) land before the CTA exits
+  __syncthreads();
+  if (warp == kProdWarp && lane == 0)
+    for (uint32_t q = seq > kStages ? seq - kStages : 0; q < seq; ++q)
+      mbar_drain(&S.full[q % kStages], (q / kStages) & 1u, a.err, 0x405u);
+}
+
+struct Layout {
+  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, seg_w, total;
+};
+
+Layout verify_layout(int B, int K, int V) {
+  const size_t nseg = (V + kSeg - 1) / kSeg, nrseg = (V + kRSeg - 1) / kRSeg;
+  const size_t rows = static_cast<size_t>(B) * (K + 1), nb = static_cast<size_t>(B);
+  Layout L{};
   size_t off = 0;
-  a.rp_m = reinterpret_cast<float*>(scratch + off);
-  off = align_up(off + rows * nseg * sizeof(float), 256);
-  a.rp_S = reinterpret_cast<double*>(scratch + off);
-  off = align_up(off + rows * nseg * sizeof(double), 256);
-  a.x_tok = reinterpret_cast<float*>(scratch + off);
-  off = align_up(off + static_cast<size_t>(a.B) * a.K * sizeof(float), 256);
-  a.seg_w = reinterpret_cast<double*>(scratch + off);
-  off = align_up(off + static_cast<size_t>(a.B) * nseg * sizeof(double), 256);
-  a.dec = reinterpret_cast<VerifyDecision*>(scratch + off);
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.rowinfo = take(rows * sizeof(RowInfo));
+  L.rowbase = take(nb * sizeof(int));
+  L.ctl = take(8 * sizeof(unsigned));
+  L.part_m = take(rows * nseg * sizeof(float));
+  L.part_S = take(rows * nseg * sizeof(double));
+  L.x_tok = take(rows * sizeof(float));
+  L.rstat = take(rows * sizeof(RowStat));
+  L.accepted = take(rows * sizeof(int));
+  L.dec = take(nb * sizeof(ResDec));
+  L.resfac = take(nb * nseg * sizeof(float2));
+  L.list = take(nb * sizeof(int));
+  L.seg_w = take(nb * nrseg * sizeof(double));
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+size_t verify_scratch_bytes(int B, int K, int V) { return verify_layout(B, K, V).total; }
+
+cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
+  Params P{};
+  P.a = a;
+  P.nseg = (a.V + kSeg - 1) / kSeg;
+  P.nrseg = (a.V + kRSeg - 1) / kRSeg;
+  P.ngrp = (a.V + kRowItem - 1) / kRowItem;
+  P.nrgrp = (a.V + kResItem - 1) / kResItem;
+  const Layout L = verify_layout(a.B, a.K, a.V);
+  P.w.rowinfo = reinterpret_cast<RowInfo*>(region + L.rowinfo);
+  P.w.rowbase = reinterpret_cast<int*>(region + L.rowbase);
+  P.w.ctl = reinterpret_cast<unsigned*>(region + L.ctl);
+  P.w.part_m = reinterpret_cast<float*>(region + L.part_m);
+  P.w.part_S = reinterpret_cast<double*>(region + L.part_S);
+  P.w.x_tok = reinterpret_cast<float*>(region + L.x_tok);
+  P.w.rstat = reinterpret_cast<RowStat*>(region + L.rstat);
+  P.w.accepted = reinterpret_cast<int*>(region + L.accepted);
+  P.w.dec = reinterpret_cast<ResDec*>(region + L.dec);
+  P.w.resfac = reinterpret_cast<float2*>(region + L.resfac);
+  P.w.list = reinterpret_cast<int*>(region + L.list);
+  P.w.seg_w = reinterpret_cast<double*>(region + L.seg_w);
 
   int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int wpc = WT / 32;
-  const long long items1 = static_cast<long long>(a.B) * (a.K + 1) * a.nseg;
-  const int g1 = static_cast<int>(std::min<long long>((items1 + wpc - 1) / wpc, static_cast<long long>(sms) * 8));
-  verify_rows_kernel<<<g1, WT, 0, stream>>>(a);
-  verify_decide_kernel<<<a.B, WT, 0, stream>>>(a);
-  const long long items2 = static_cast<long long>(a.B) * a.nseg;
-  const int g2 = static_cast<int>(std::min<long long>((items2 + wpc - 1) / wpc, static_cast<long long>(sms) * 8));
-  verify_segsum_kernel<<<g2, WT, 0, stream>>>(a);
-  verify_final_kernel<<<(a.B + wpc - 1) / wpc, WT, 0, stream>>>(a);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const size_t smem = static_cast<size_t>(kStages) * kStageBytes + sizeof(Smem);
+  e = cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  verify_plan_kernel<<<1, kPlanThreads, 0, stream>>>(P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long rows = static_cast<long long>(a.B) * (a.K + 1);
+  const long long units = std::max(rows * P.ngrp, (rows + kWarps - 1) / kWarps);
+  const int G = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, units)));
+  // cooperative, and allowed to start while the plan kernel runs
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, verify_kernel, P);
+  if (e == cudaErrorNotSupported) {  // without the early start
+    (void)cudaGetLastError();
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, verify_kernel, P);
+  }
+  return e;
 }
 
 }  // namespace dspark
