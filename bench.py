@@ -17,6 +17,7 @@ full batch); it is the baseline arm, not a GPU implementation.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -126,6 +127,31 @@ def cpu_baseline(inp: dict, seconds: float = 15.0) -> dict:
                       f"schedule on the full batch), scaled by {B}/{n_req}; {spent:.1f} s of CPU work"}
 
 
+def source_digest() -> str:
+    """sha256 over the library's CUDA sources: a recorded DRAM traffic figure is
+    only reported while the kernels are the ones it was measured on."""
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "speculative_decoding_semi_b200", "csrc")
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(src, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str) -> dict:
+    """DRAM bytes (read + write) per launch of each kernel, from the ncu capture
+    recorded in profiles/traffic.json, or {} when the sources have changed."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        tj = json.load(f)
+    if tj.get("workload") != workload or tj.get("source_sha256") != source_digest():
+        return {}
+    return {k: v for k, v in tj.get("dram_bytes_per_launch", {}).items()}
+
+
 def draft_bytes(B, K, V, r, factor_bytes):
     """Algorithmic HBM bytes of one draft launch: base read + z write + Bf once
     + gathered A rows + per-position outputs."""
@@ -194,7 +220,7 @@ def run_gpu(args):
     bufs = rnd.RoundBuffers(B, K, V, r)
     stream = torch.cuda.Stream()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-    launches_per_round = 1 + 2 + 3  # draft, schedule (rank, final), verify (rows, decide, final)
+    launches_per_round = 1 + 2 + 2  # draft, schedule (rank, final), verify (plan, main)
 
     def one_round(ev=None):
         with torch.cuda.stream(stream):
@@ -290,13 +316,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(inp, seconds=args.cpu_seconds)
 
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            tj = json.load(f)
-        if tj.get("workload") == w.name and tj.get("kernel_version") == "draft-generic-v1":
-            traffic = tj.get("draft_bytes_per_launch")
+    traffic = measured_traffic(w.name)
     line = {
         "metric": "draft+schedule+verify rounds/sec", "value": value, "unit": "rounds/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
@@ -310,9 +330,11 @@ def run_gpu(args):
                      "p90": float(np.percentile(t_round, 90))},
         "roofline": {"bound": "hbm", "kernel": "dspark_markov_draft", "achieved": draft_gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": draft_gbs / peaks["hbm_gbs"],
-                     "traffic": traffic, "algorithmic_bytes": dbytes, "peak_source": peaks["source"]},
+                     "traffic": traffic.get("draft_tc_kernel"), "algorithmic_bytes": dbytes,
+                     "peak_source": peaks["source"]},
         "roofline_verify": {"bound": "hbm", "achieved": verify_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": verify_gbs / peaks["hbm_gbs"], "algorithmic_bytes": vbytes},
+                            "frac": verify_gbs / peaks["hbm_gbs"], "traffic": traffic.get("verify_kernel"),
+                            "algorithmic_bytes": vbytes},
         "round_stats": {"verify_tokens": int((L + 1).sum()), "accepted_mean": float(acc.mean()),
                         "emitted_per_round": int(n_out.sum())},
         "gpu_launches": launches_per_round * args.steps,

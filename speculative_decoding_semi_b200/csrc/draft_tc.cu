@@ -283,7 +283,10 @@ __device__ __forceinline__ int warp_search(int n, Get get, Thr thr_of, int lane,
   const bool in_regs = per <= kSearchRegs;
   if (in_regs) {
 #pragma unroll
-    for (int j = 0; j < kSearchRegs; ++j) vals[j] = (lo + j < hi) ? get(lo + j) : 0.0;
+    for (int j = 0; j < kSearchRegs; ++j) vals[j] = get(min(lo + j, n - 1));  // clamped: the loads issue together
+#pragma unroll
+    for (int j = 0; j < kSearchRegs; ++j)
+      if (lo + j >= hi) vals[j] = 0.0;
 #pragma unroll
     for (int j = 0; j < kSearchRegs; ++j) {
       local += vals[j];
@@ -356,6 +359,69 @@ __device__ __forceinline__ int warp_search(int n, Get get, Thr thr_of, int lane,
   return best;
 }
 
+// exp(z): the weight of the epilogue's slice sums and of the selector's rescan.
+__device__ __forceinline__ float zw(float z) { return expf(z); }
+
+// First element of zc[0..n) (n a multiple of 32; one warp) whose running fp64
+// sum of the weights exp(z) exceeds R with a positive weight, or -1 (*last
+// then gives the last positive one). In chunks of 1024, lane l owns the 32
+// consecutive elements at 32 l: its loads issue together, one warp-wide scan
+// over the lanes' totals locates the lane, which searches its own elements.
+__device__ int scan_slice(const float* zc, int n, int lane, double R, int* last, double* w_hit) {
+  double before = 0.0;
+  int found = -1, lastp = -1;
+  *w_hit = 0.0;
+  for (int c0 = 0; c0 < n && found < 0; c0 += 1024) {
+    const int e0 = c0 + 32 * lane;
+    const bool mine = e0 < n;  // all 32 elements or none, since n % 32 == 0
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      v[k] = mine ? __ldcg(reinterpret_cast<const float4*>(zc + e0 + 4 * k)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    double w[32];
+    double lsum = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      w[4 * k] = mine ? static_cast<double>(zw(v[k].x)) : 0.0;
+      w[4 * k + 1] = mine ? static_cast<double>(zw(v[k].y)) : 0.0;
+      w[4 * k + 2] = mine ? static_cast<double>(zw(v[k].z)) : 0.0;
+      w[4 * k + 3] = mine ? static_cast<double>(zw(v[k].w)) : 0.0;
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) lsum += w[e];
+    const double inc = warp_inclusive_scan(lsum);
+    double ex = __shfl_up_sync(0xffffffffu, inc, 1);
+    if (lane == 0) ex = 0.0;
+    ex += before;
+    int hit = -1, lp = -1;
+    double wh = 0.0;
+    if (ex + lsum > R) {
+      double c = ex;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        if (hit < 0 && w[e] > 0.0 && c + w[e] > R) {
+          hit = e;
+          wh = w[e];
+        }
+        c += w[e];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (w[e] > 0.0) lp = e0 + e;
+    lastp = max(lastp, warp_max_int(lp));
+    const unsigned hits = __ballot_sync(0xffffffffu, hit >= 0);
+    if (hits) {
+      const int hl = __ffs(hits) - 1;
+      found = c0 + 32 * hl + __shfl_sync(0xffffffffu, hit, hl);
+      *w_hit = __shfl_sync(0xffffffffu, wh, hl);
+    }
+    before += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  *last = lastp;
+  return found;
+}
+
 // Draw request b's token at position i (one warp). Writes draft_tokens,
 // q_tok and lse_q; returns the token.
 __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane) {
@@ -374,25 +440,16 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
   float shift = 0.f;
   if (W >= 1e-30 && W <= 1e30) {
     const double R = u * W - ex;
-    // level 2: the slice's own weights exp(z), read as coalesced rows of 128
-    // (lane l holds elements 4l..4l+3 of each row) and scanned in vocabulary
-    // order: rows in turn, lanes in turn, then the lane's four elements
+    // level 2: the slice's own weights exp(z), in vocabulary order
     int lo, hi, x, last;
     chunk_bounds(d.V, kUnit, G, c, &lo, &hi);
-    const int n = hi - lo;
     const float* zc = zrow + lo;
-    x = scan_rows128<12, float4>(
-        n, lane, R, [&](int e) { return __ldcg(reinterpret_cast<const float4*>(zc + e)); },
-        [&](const float4& v, double(&w)[4]) {
-          w[0] = static_cast<double>(expf(v.x));
-          w[1] = static_cast<double>(expf(v.y));
-          w[2] = static_cast<double>(expf(v.z));
-          w[3] = static_cast<double>(expf(v.w));
-        },
-        &last);
-    if (x < 0) x = max(last, 0);  // rounding: the last positive weight
+    x = scan_slice(zc, hi - lo, lane, R, &last, &w_t);
+    if (x < 0) {  // rounding: the last positive weight
+      x = max(last, 0);
+      w_t = static_cast<double>(zw(__ldcg(zc + x)));
+    }
     tok = lo + x;
-    w_t = static_cast<double>(expf(__ldcg(zc + x)));
   } else {
     // the whole row with its exact maximum as the shift
     float mx = -INFINITY;
@@ -773,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < kChunk; ++c) {
                       const float zz = box[c * kUnit + lane] + __uint_as_float(rg[c]);
                       box[c * kUnit + lane] = zz;
-                      cacc[c] += (col0 + c < nreal) ? static_cast<double>(expf(zz)) : 0.0;
+                      cacc[c] += (col0 + c < nreal) ? static_cast<double>(zw(zz)) : 0.0;
                     }
                   } else {
 #pragma unroll
@@ -784,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int cc = half * 16 + c;
                         const float zz = box[cc * kUnit + lane] + __uint_as_float(rg[cc]);
                         box[cc * kUnit + lane] = zz;
-                        w[c] = (col0 + cc < nreal) ? static_cast<double>(expf(zz)) : 0.0;
+                        w[c] = (col0 + cc < nreal) ? static_cast<double>(zw(zz)) : 0.0;
                       }
                       acc[2 * kk + half] += reduce16(w, lane);
                     }

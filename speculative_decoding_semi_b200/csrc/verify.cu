@@ -230,29 +230,27 @@ __global__ void __launch_bounds__(kPlanThreads) verify_plan_kernel(Params p) {
 }
 
 // ------------------------------------------------------ warp-level helpers
-// Inverse CDF over nseg segment weights (one warp; `weight(q)` must return the
-// same value whenever called): the first segment whose inclusive running sum
-// exceeds u * total with a positive weight, else (rounding) the last positive
-// one. Lane l owns a contiguous block of segments. *rem = u * total minus the
-// weight before the chosen segment. Returns -1 if total <= 0.
-template <class Weight>
-__device__ int pick_segment(int nseg, float u, int lane, Weight weight, double* rem) {
+// Inverse CDF over nseg segment weights, one warp; lane l owns the segments
+// [l per, l per + per). raw(q) loads what segment q's weight needs and
+// value(raw) computes the weight (the same value whenever called); the N <=
+// per-lane raw values are loaded before any is used, so their loads issue
+// together. Returns the first segment whose inclusive running sum exceeds
+// u * total with a positive weight, else (rounding) the last positive one,
+// with *rem = u * total minus the weight before it; -1 if total <= 0.
+template <int N, class Raw, class Value>
+__device__ int pick_segment_n(int nseg, float u, int lane, Raw raw, Value value, double* rem) {
   const int per = (nseg + 31) / 32;
   const int lo = min(nseg, lane * per), hi = min(nseg, lo + per);
-  const bool cached = per <= kRegWeight;
-  double wv[kRegWeight];
+  using T = decltype(raw(0));
+  T rv[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) rv[i] = raw(min(lo + i, nseg - 1));  // clamped: always a valid address
+  double wv[N];
   double local = 0.0;
-  if (cached) {
-    // unconditional calls on clamped indices, so that every load issues at once
 #pragma unroll
-    for (int i = 0; i < kRegWeight; ++i) wv[i] = weight(min(lo + i, nseg - 1));
-#pragma unroll
-    for (int i = 0; i < kRegWeight; ++i) {
-      if (lo + i >= hi) wv[i] = 0.0;
-      local += wv[i];
-    }
-  } else {
-    for (int q = lo; q < hi; ++q) local += weight(q);
+  for (int i = 0; i < N; ++i) {
+    wv[i] = lo + i < hi ? value(rv[i]) : 0.0;
+    local += wv[i];
   }
   const double inc = warp_inclusive_scan(local);
   double ex = __shfl_up_sync(0xffffffffu, inc, 1);
@@ -262,7 +260,53 @@ __device__ int pick_segment(int nseg, float u, int lane, Weight weight, double* 
   const double thr = static_cast<double>(u) * total;
   int cand = INT_MAX, lastq = -1;
   double cand_ex = 0.0, last_ex = 0.0, c = ex;
-  auto visit = [&](int q, double v) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const double v = wv[i];
+    if (v > 0.0) {
+      if (cand == INT_MAX && c + v > thr) {
+        cand = lo + i;
+        cand_ex = c;
+      }
+      lastq = lo + i;
+      last_ex = c;
+    }
+    c += v;
+  }
+  int seg = warp_min_int(cand);
+  double seg_ex;
+  if (seg != INT_MAX) {
+    seg_ex = __shfl_sync(0xffffffffu, cand_ex, seg / per);
+  } else {
+    seg = warp_max_int(lastq);
+    if (seg < 0) return -1;
+    seg_ex = __shfl_sync(0xffffffffu, last_ex, seg / per);
+  }
+  *rem = thr - seg_ex;
+  return seg;
+}
+
+// The same for any nseg: the smallest register block that holds per, or a
+// plain loop beyond 32 segments per lane.
+template <class Raw, class Value>
+__device__ int pick_segment(int nseg, float u, int lane, Raw raw, Value value, double* rem) {
+  const int per = (nseg + 31) / 32;
+  if (per <= 4) return pick_segment_n<4>(nseg, u, lane, raw, value, rem);
+  if (per <= 8) return pick_segment_n<8>(nseg, u, lane, raw, value, rem);
+  if (per <= 16) return pick_segment_n<16>(nseg, u, lane, raw, value, rem);
+  const int lo = min(nseg, lane * per), hi = min(nseg, lo + per);
+  double local = 0.0;
+  for (int q = lo; q < hi; ++q) local += value(raw(q));
+  const double inc = warp_inclusive_scan(local);
+  double ex = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) ex = 0.0;
+  const double total = __shfl_sync(0xffffffffu, inc, 31);
+  if (!(total > 0.0)) return -1;
+  const double thr = static_cast<double>(u) * total;
+  int cand = INT_MAX, lastq = -1;
+  double cand_ex = 0.0, last_ex = 0.0, c = ex;
+  for (int q = lo; q < hi; ++q) {
+    const double v = value(raw(q));
     if (v > 0.0) {
       if (cand == INT_MAX && c + v > thr) {
         cand = q;
@@ -272,13 +316,6 @@ __device__ int pick_segment(int nseg, float u, int lane, Weight weight, double* 
       last_ex = c;
     }
     c += v;
-  };
-  if (cached) {
-#pragma unroll
-    for (int i = 0; i < kRegWeight; ++i)
-      if (lo + i < hi) visit(lo + i, wv[i]);
-  } else {
-    for (int q = lo; q < hi; ++q) visit(q, weight(q));
   }
   int seg = warp_min_int(cand);
   double seg_ex;
@@ -387,25 +424,27 @@ __device__ void row_stats(const Params& P, int R, int lane) {
 }
 
 // Draw from p of compact row R (the bonus row, or a rejected row whose
-// residual vanished) with the row pass's segment sums; one warp.
-__device__ __noinline__ int sample_p(const Params& P, int R, float u, int lane) {
+// residual vanished) with the row pass's segment sums; one warp. With `warm`
+// set it runs its whole path on whatever the arrays hold, to load its code
+// into the SM's instruction cache ahead of the phase that needs it.
+__device__ __noinline__ int sample_p(const Params& P, int R, float u, int lane, bool warm = false) {
   const VerifyArgs& a = P.a;
   const float* pm = P.w.part_m + static_cast<long long>(R) * P.nseg;
   const double* pS = P.w.part_S + static_cast<long long>(R) * P.nseg;
-  const double M = __ldcg(&P.w.rstat[R].M), W = __ldcg(&P.w.rstat[R].W);
+  const double M = __ldcg(&P.w.rstat[R].M);
   const long long row = P.w.rowinfo[R].row;
-  auto weight = [&](int q) -> double {
-    const double S = __ldcg(pS + q);
-    const float h = __ldcg(pm + q);
-    return S > 0.0 ? __dmul_rn(S, seg_scale(h, M) / W) : 0.0;
-  };
+  // segment weights S 2^(h - M): the row's total W scales them all alike and
+  // cancels in the inverse CDF
   double rem = 0.0;
-  const int seg = pick_segment(P.nseg, u, lane, weight, &rem);
-  if (seg < 0) return 0;  // no positive weight: degenerate row
-  const float m_s = __ldcg(pm + seg);
-  const double Rs = rem / (seg_scale(m_s, M) / W);
-  const float* x = a.target + row * a.V + static_cast<long long>(seg) * kSeg;
-  const int n = min(kSeg, a.V - seg * kSeg);
+  const int seg = pick_segment(
+      P.nseg, u, lane, [&](int q) { return make_double2(__ldcg(pS + q), static_cast<double>(__ldcg(pm + q))); },
+      [&](double2 r) { return r.x > 0.0 ? __dmul_rn(r.x, seg_scale(static_cast<float>(r.y), M)) : 0.0; }, &rem);
+  if (seg < 0 && !warm) return 0;  // no positive weight: degenerate row
+  const int sg = max(seg, 0);
+  const float m_s = __ldcg(pm + sg);
+  const double Rs = rem / seg_scale(m_s, M);
+  const float* x = a.target + row * a.V + static_cast<long long>(sg) * kSeg;
+  const int n = min(kSeg, a.V - sg * kSeg);
   constexpr int E = kSeg / 32;
   float w[E];
 #pragma unroll
@@ -420,7 +459,7 @@ __device__ __noinline__ int sample_p(const Params& P, int R, float u, int lane) 
   int last = -1;
   int k = rescan<E>(n, lane, Rs, w, &last);
   if (k < 0) k = max(last, 0);
-  return seg * kSeg + k;
+  return sg * kSeg + k;
 }
 
 // Emits request b's accepted drafts and the drawn token.
@@ -481,13 +520,15 @@ __device__ __noinline__ void decide(const Params& P, int b, int lane) {
 }
 
 // Phase 5, one warp: the resampled token of listed request b.
-__device__ __noinline__ void resample(const Params& P, int b, int lane) {
+// The resampled token of request b from its residual segment sums; `warm`
+// as for sample_p.
+__device__ __noinline__ int residual_token(const Params& P, int b, const ResDec& d, float u, int lane, bool warm) {
   const VerifyArgs& a = P.a;
-  const ResDec d = P.w.dec[b];
   const double* sw = P.w.seg_w + static_cast<long long>(b) * P.nrseg;
-  const float u = a.u_resample[b];
   double rem = 0.0;
-  const int seg = pick_segment(P.nrseg, u, lane, [&](int q) -> double { return __ldcg(sw + q); }, &rem);
+  int seg = pick_segment(
+      P.nrseg, u, lane, [&](int q) { return __ldcg(sw + q); }, [](double v) { return v; }, &rem);
+  if (warm) seg = max(seg, 0);
   int tok;
   if (seg < 0) {
     tok = sample_p(P, d.R, u, lane);  // the residual vanished (rounding): draw from p
@@ -514,7 +555,12 @@ __device__ __noinline__ void resample(const Params& P, int b, int lane) {
     if (k < 0) k = max(last, 0);
     tok = static_cast<int>(v0) + k;
   }
-  write_output(P, b, d.acc, tok, lane);
+  return tok;
+}
+
+__device__ __noinline__ void resample(const Params& P, int b, int lane) {
+  const ResDec d = P.w.dec[b];
+  write_output(P, b, d.acc, residual_token(P, b, d, P.a.u_resample[b], lane, false), lane);
 }
 
 // -------------------------------------------------------- consumer bodies
@@ -621,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
   float* stages = reinterpret_cast<float*>(smem);
   Smem& S = *reinterpret_cast<Smem*>(smem + kStages * kStageBytes);
   __shared__ int s_flag;
+  __shared__ volatile int s_sink;
   const VerifyArgs& a = P.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -713,6 +760,19 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
         bulk_load(dst, a.target + ri.row * a.V + v0, bytes, full);
       },
       [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_row(P, ds, stage, empty, w, lane); });
+  // the spare warps run the later phases' code once while the rows stream, so
+  // that those phases do not start on a cold instruction cache
+  if (warp > kProdWarp && n_rows > 0) {
+    int r = 0;
+    if (warp == kProdWarp + 1) r = sample_p(P, 0, 0.5f, lane, true);
+    if (warp == kProdWarp + 2) {
+      ResDec d{};
+      d.row = P.w.rowinfo[0].row;
+      r = residual_token(P, 0, d, 0.5f, lane, true);
+    }
+    if (warp == kProdWarp + 3) row_stats(P, 0, lane);  // rewritten in phase 2
+    if (lane == 0) s_sink = r;
+  }
   ok = __syncthreads_and(ok) && grid_barrier(P, 0, &s_flag);
 
   // ---- phase 2: row statistics and accept tests
