@@ -39,6 +39,9 @@ def test_tiny_many_seeds():
     (1, dict(B=3, K=2, V=96, r=256, n_prof=16)),
     (1, dict(B=17, K=4, V=4096, r=192, n_prof=80)),
     (1, dict(B=64, K=3, V=151936, r=256, n_prof=2048)),
+    # request groups of unequal size (32 + 16; 64 + 32, three chunks in the first)
+    (1, dict(B=48, K=4, V=8192, r=64, n_prof=256)),
+    (1, dict(B=96, K=3, V=16384, r=256, n_prof=512)),
     # K = 32: verify lengths of 32 (33 target rows per request)
     (1, dict(B=3, K=32, V=2048, r=64, n_prof=128)),
     (0, dict(B=2, K=32, V=1024, r=16, n_prof=80)),
