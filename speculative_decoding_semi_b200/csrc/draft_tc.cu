@@ -389,11 +389,11 @@ __device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t,
 }
 
 // One warp: every lane waits for *ctr >= target (bounded), so the warp stays
-// converged for the collective code that follows.
+// converged for the collective code that follows. Each lane's own acquire load
+// of the counter orders its later reads; no further fence is needed.
 __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned target, unsigned* err,
                                                   unsigned where, volatile int* abort, int lane) {
   const bool ok = __all_sync(0xffffffffu, wait_at_least(ctr, target, err, where));
-  __threadfence();
   if (!ok && lane == 0) *abort = 1;
   return ok;
 }
@@ -577,7 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
       }
     }
-    __threadfence();
+    // Publishing: the warp barrier orders every lane's writes before lane 0's
+    // release reduction, which makes them visible at gpu scope (on an SM with
+    // copies in flight a separate gpu fence costs microseconds).
     __syncwarp();
     for (int gr = 0; gr < p.ngroups; ++gr) {
       const int gbase = gr * p.gsize, nreal = group_real(p, gr);
@@ -604,7 +606,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           d.part_S[static_cast<long long>(gbase + n) * G + g] = S;
           d.part_m[static_cast<long long>(gbase + n) * G + g] = 0.f;
         }
-        __threadfence();
         __syncwarp();
         const unsigned slot = static_cast<unsigned>(i * p.ngroups + gr);
         if (lane == 0) red_release_gpu_add(&p.sync_part[slot], 1u);
@@ -622,7 +623,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (i + 1 < d.K) {
           const unsigned nslot = static_cast<unsigned>((i + 1) * p.ngroups + gr);
-          __threadfence();
           __syncwarp();
           if (lane == 0 && mine) red_release_gpu_add(&p.sync_tok[nslot], mine);
           ok = warp_wait_counter(&p.sync_tok[nslot], static_cast<unsigned>(nreal), d.err, 0x700u + nslot, s_abort,
@@ -677,7 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_all();
       }
-      __threadfence();
+      // the stores are complete; the warp barrier and the mbarrier's release
+      // hand them, with the lanes' unit sums, to the selector, whose gpu-scope
+      // release reduction publishes them
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.step_done[pending]);
       pending = -1;

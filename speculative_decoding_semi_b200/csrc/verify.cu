@@ -650,12 +650,13 @@ struct Smem {
 // to every thread after it. Called between streaming phases, with no copy in
 // flight.
 __device__ bool grid_barrier(const Params& P, int k, int* s_flag) {
+  // The CTA barrier orders every thread's writes before thread 0's release
+  // reduction (gpu scope), and thread 0's acquire loads before every thread's
+  // later reads; separate gpu fences would only add microseconds.
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
     red_release_gpu_add(P.w.ctl + kCtlBar + k, 1u);
     const bool ok = wait_at_least(P.w.ctl + kCtlBar + k, gridDim.x, P.a.err, 0x500u + k);
-    __threadfence();
     *s_flag = ok ? 1 : 0;
   }
   __syncthreads();
