@@ -466,10 +466,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               }
               uint8_t* dst = smem + Ly.bf + stage * kBfStageBytes;
-              const int v0 = lo + phys_tile(i, gr, p.ngroups, ntiles, t) * kTileRows;
-              mbar_arrive_expect_tx(&bars.bf_full[stage], kBfStageBytes);
+              const int pt = phys_tile(i, gr, p.ngroups, ntiles, t);
+              const int v0 = lo + pt * kTileRows;
+              // a last tile of at most 64 rows needs only the first 64-row box:
+              // the MMA's rows beyond it are never read by the epilogue
+              const bool both = (pt == ntiles - 1 ? last_rows : kTileRows) > 64;
+              mbar_arrive_expect_tx(&bars.bf_full[stage], both ? kBfStageBytes : kBfBoxBytes);
               tma_load_2d(dst, &tm_bf, v0, s * kKStage, &bars.bf_full[stage], pol);
-              tma_load_2d(dst + kBfBoxBytes, &tm_bf, v0 + 64, s * kKStage, &bars.bf_full[stage], pol);
+              if (both) tma_load_2d(dst + kBfBoxBytes, &tm_bf, v0 + 64, s * kKStage, &bars.bf_full[stage], pol);
               issued[stage] = true;
               issued_parity[stage] = phase;
               if (++stage == p.nbf) {
