@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 
 def test_tiny_many_seeds():
     t = parity.Tally()
-    for seed in range(40):
+    for seed in range(500):
         inp = synth.make_round(0, seed=5000 + seed)
         parity.check_round(inp, tally=t)
     t.check()
@@ -113,6 +113,20 @@ def test_full_size_workloads(key, sample):
     B = inp["base"].shape[0]
     reqs = None if sample is None else np.linspace(0, B - 1, sample).astype(int)
     t, g = parity.check_round(inp, requests=reqs, check_z=sample is None)
+    t.check()
+
+
+@pytest.mark.parametrize("key,seeds,sample", [("qwen3", 4, None), ("latency", 20, None), ("highconc", 3, 8),
+                                             ("mixed", 3, 8)])
+def test_full_size_seed_volume(key, seeds, sample):
+    """More seeds of every full-size workload, the excused near-ties pooled
+    over them (z itself is compared in test_full_size_workloads)."""
+    t = parity.Tally()
+    for k in range(seeds):
+        inp = synth.make_round(key, seed=7000 + k)
+        B = inp["base"].shape[0]
+        reqs = None if sample is None else np.linspace(0, B - 1, sample).astype(int)
+        parity.check_round(inp, requests=reqs, tally=t, check_z=False)
     t.check()
 
 
