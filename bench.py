@@ -52,6 +52,24 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of x over all ranks of the process group (x itself when
+    there is one rank): every multi-GPU time is the slowest rank's."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, slowest_ms: float) -> float:
+    """Units all ranks processed per second over the slowest rank's time
+    (replicas: every rank runs the same number of units)."""
+    return units_per_rank * world / (slowest_ms / 1000.0)
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running."""
 
@@ -262,13 +280,8 @@ def run_gpu(args):
     t_sched = [e[1].elapsed_time(e[2]) for e in evs]
     t_ver = [e[2].elapsed_time(e[3]) for e in evs]
     t_round = [a + b + c for a, b, c in zip(t_draft, t_sched, t_ver)]
-    total_ms = sum(t_round)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-    rounds_total = args.steps * world
-    value = rounds_total / (total_ms / 1000.0)
+    total_ms = max_over_ranks(sum(t_round), world, device="cuda")
+    value = whole_job_rate(args.steps, world, total_ms)
 
     L = bufs.verify_len.cpu().numpy()
     acc = bufs.accepted.cpu().numpy()
@@ -307,12 +320,8 @@ def run_gpu(args):
                 out_host[B * (K + 1):].copy_(bufs.n_out.view(-1), non_blocking=True)
             ev1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = ev0.elapsed_time(ev1)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": e2e_steps * world / (e2e_ms / 1000.0), "unit": "rounds/s",
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, device="cuda")
+        e2e = {"value": whole_job_rate(e2e_steps, world, e2e_ms), "unit": "rounds/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "note": "Markov factors are model weights kept resident; per-round logits, confidences "
                        "and uniforms are copied in, emitted tokens copied out"}
