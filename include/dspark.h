@@ -162,9 +162,12 @@ dspark_status dspark_schedule_static(const float* conf_logits, const float* temp
  * for persisting accesses (cudaLimitPersistingL2CacheSize, capped at the
  * device's maximum); *granted (if non-NULL) receives the size in effect. The
  * draft kernel reads the Markov factor Bf with an L2 evict-last hint at every
- * position, and such lines are only kept in this set-aside, which is empty by
- * default. The setting belongs to the calling process's CUDA context and
- * ends with it; call once at set-up, outside stream capture. */
+ * position; a set-aside reserves capacity for such lines at the expense of the
+ * rest of the L2. It is empty by default, and on B200 the qwen3-sized draft
+ * ran slower with one than without (the logits streamed through L2 need the
+ * capacity), so the library never requests one itself. The setting belongs to
+ * the calling process's CUDA context and ends with it; call once at set-up,
+ * outside stream capture. */
 dspark_status dspark_l2_reserve(size_t bytes, size_t* granted);
 
 /* Synchronise `stream`, return the status recorded in the workspace's error
