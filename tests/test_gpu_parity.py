@@ -4,7 +4,7 @@ Sizes: the tiny workload over many seeds; medium sizes that span many
 vocabulary chunks and verify segments with ragged tails (V not a multiple of
 the 4096-wide segment); every full-size workload (all requests where the
 oracle is quick, a sample of requests otherwise); the exhaustive V=8
-enumeration; and edge cases (B=1, K=1, V=8, every verify length 0, packed
+enumeration; and edge cases (B=1, K=1, V=8, every verify length 0, extreme logits, packed
 ragged target rows, invalid indices reported through the error word).
 """
 import numpy as np
@@ -127,6 +127,26 @@ def test_full_size_seed_volume(key, seeds, sample):
         B = inp["base"].shape[0]
         reqs = None if sample is None else np.linspace(0, B - 1, sample).astype(int)
         parity.check_round(inp, requests=reqs, tally=t, check_z=False)
+    t.check()
+
+
+@pytest.mark.parametrize("like", [0, 1])
+def test_extreme_logits_take_the_shifted_paths(like):
+    """Rows whose sum of exp(z) leaves the fixed-shift range: the draft
+    redraws them with the exact maximum, verify sums those segments with
+    their own shift (fp32 and bf16 factors: both draft kernels)."""
+    w = synth.custom(like, B=6, K=4, V=8192, r=64, n_prof=64)
+    t = parity.Tally()
+    for seed in range(2):
+        inp = synth.make_round(w, seed=900 + seed)
+        base = inp["base"].copy()
+        tgt = inp["target"].copy()
+        base[0] += 90.0      # exp(z) overflows fp32 for the whole row
+        base[1, 1] -= 150.0  # underflows at one position
+        tgt[2] += 90.0       # verify segments above the fixed-shift range
+        tgt[3, 0] -= 150.0   # and below it
+        inp["base"], inp["target"] = base, tgt
+        parity.check_round(inp, tally=t)
     t.check()
 
 
