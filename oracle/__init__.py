@@ -17,10 +17,13 @@ The pages state each step in words only; where they leave a detail open the
 reading taken is named in the function's docstring.
 
 Pins (tests/test_oracle_*.py): exhaustive enumeration at V=8 that the verified
-output is distributed exactly as the target; zero Markov factors reduce the
-draft to independent per-position inverse-CDF sampling; the bias equals a
-brute-force fp64 triple loop; the scheduler equals brute force over every
-length assignment; survival has closed forms at c=0 and c -> +-inf.
+output is distributed exactly as the target; factors that force each draft
+token to be a fixed function of the previous one (the chain, with and without
+teacher forcing); forced acceptance counts that fix which row the final token
+comes from; zero Markov factors reduce the draft to independent per-position
+inverse-CDF sampling; the bias equals a brute-force fp64 triple loop; the
+scheduler equals brute force over every length assignment; survival has
+closed forms at c=0 and c -> +-inf.
 """
 from __future__ import annotations
 

@@ -17,8 +17,6 @@ import itertools
 
 import numpy as np
 
-import oracle
-
 V, K, R = 8, 3, 2
 
 
@@ -32,6 +30,29 @@ def _mid_f32(lo, hi):
     m = np.float32((lo + hi) / 2.0)
     assert lo <= float(m) < hi, (lo, hi, m)
     return m
+
+
+def _draft_q(prob, paths):
+    """Draft distributions along every path, built here without the oracle:
+    position i (0-based) is corrected by the token before it (the anchor at
+    i = 0) with the bias summed term by term in fp64, then softmaxed. The
+    uniforms placed at the midpoints of these intervals are what makes the
+    oracle's own chain (oracle.draft without teacher forcing) checkable
+    against the paths."""
+    A = prob["A"].astype(np.float64)
+    Bf = prob["Bf"].astype(np.float64)
+    n = len(paths)
+    q = np.empty((n, K, V))
+    for pi in range(n):
+        prev = int(prob["anchor"])
+        for i in range(K):
+            z = prob["base"][i].astype(np.float64).copy()
+            for v in range(V):
+                for k in range(R):
+                    z[v] += A[prev, k] * Bf[k, v]
+            q[pi, i] = _softmax(z)
+            prev = int(paths[pi, i])
+    return q
 
 
 def make_problem(seed=7, factor_std=0.7):
@@ -54,14 +75,13 @@ def build_batch(prob, L):
     """All pieces for verify length L (0 <= L <= K).
 
     Returns a dict of batch arrays (one row per piece) plus `weight` [N] and
-    `q` [N,K,V] (the oracle's draft distributions along each path).
+    `q` [N,K,V] (the draft distributions along each path, built without the oracle).
     """
     paths = np.array(list(itertools.product(range(V), repeat=K)), np.int64)  # [512,K]
     n = len(paths)
     base = np.broadcast_to(prob["base"], (n, K, V)).copy()
     anchor = np.full(n, prob["anchor"], np.int32)
-    d = oracle.draft(base, prob["A"], prob["Bf"], anchor, np.zeros((n, K), np.float32), teacher=paths)
-    q = oracle.softmax(d["z"])  # [n,K,V], q[:, i] = q_{i+1}(. | t_i)
+    q = _draft_q(prob, paths)  # [n,K,V], q[:, i] = q_{i+1}(. | t_i)
     rows = {k: [] for k in ("path", "u_draft", "u_accept", "u_resample", "weight", "target", "q")}
     for pi in range(n):
         path = paths[pi]

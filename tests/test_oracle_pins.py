@@ -1,7 +1,13 @@
 """Pins of the CPU oracle to facts that do not come from the oracle itself.
 
 - losslessness: exhaustive enumeration at V=8 (the pages' claim that
-  verification keeps the target distribution exactly);
+  verification keeps the target distribution exactly), with the draft
+  intervals built independently of the oracle so that its chain is checked;
+- the draft's chain across positions: factors that force t_i = f(t_{i-1})
+  (the bias comes from the previous token, the anchor at position 1), with
+  and without teacher forcing, and planted mistakes that must fail;
+- verification with forced acceptance counts: the final token comes from the
+  row after the accepted prefix, through max(0, p - q) or the bonus row;
 - zero Markov factors reduce the draft to independent per-position sampling
   (numpy searchsorted on a scipy softmax);
 - the bias equals a brute-force fp64 triple loop;
@@ -246,3 +252,184 @@ def test_verify_special_cases():
         cdf = np.cumsum(p)
         assert v["final"][b] == np.searchsorted(cdf, float(ur[b]) * cdf[-1], side="right")
         assert np.array_equal(v["out_tokens"][b, :L[b]], tokens[b, :L[b]])
+
+
+# ---------------------------------------------------------------------------
+# The draft's chain across positions. QbitAI article, section "a cheaper
+# sequential module: the Markov head": the correction at a position depends on
+# the token drawn just before it. Factors at the tiny workload's sizes (V=1024,
+# r=32) are built so that A[t] . Bf adds +60 at exactly one token f(t) and 0
+# everywhere else; with base logits ~N(0,2) that token then holds all but
+# ~1e-20 of the mass, so any uniform in (0.001, 0.999) draws it and the chain
+# is forced: t_1 = f(anchor), t_i = f(t_{i-1}).
+CV, CR, CK, CB = 1024, 32, 6, 5
+
+
+def _chain_target(k):
+    """f's value for rank slot k: a token whose slot is k + 1 (mod r), so f
+    iterated from any anchor walks through distinct tokens."""
+    return CR * ((7 * k + 3) % CR) + (k + 1) % CR
+
+
+def _chain_factors():
+    A = np.zeros((CV, CR), np.float32)
+    A[np.arange(CV), np.arange(CV) % CR] = 60.0          # A[t] = 60 e_{t mod r}
+    Bf = np.zeros((CR, CV), np.float32)
+    Bf[np.arange(CR), [_chain_target(k) for k in range(CR)]] = 1.0
+    return A, Bf
+
+
+def _f(t):
+    return _chain_target(int(t) % CR)
+
+
+def _chain_inputs(seed):
+    rng = np.random.default_rng(seed)
+    base = rng.normal(0, 2, size=(CB, CK, CV)).astype(np.float32)
+    u = rng.uniform(0.001, 0.999, size=(CB, CK)).astype(np.float32)
+    anchor = rng.integers(0, CV, size=CB).astype(np.int32)
+    return base, u, anchor
+
+
+def _expected_chain(anchor):
+    out = np.empty((len(anchor), CK), np.int64)
+    for b, a in enumerate(anchor):
+        t = int(a)
+        for i in range(CK):
+            t = _f(t)
+            out[b, i] = t
+    return out
+
+
+def _check_chain(d, base, anchor):
+    exp = _expected_chain(anchor)
+    assert np.array_equal(d["t"], exp)
+    assert np.all(np.abs(d["q_tok"] - 1.0) < 1e-12)
+    for b in range(CB):
+        for i in range(CK):
+            assert abs(d["lse"][b, i] - (60.0 + float(base[b, i, exp[b, i]]))) < 1e-12
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_draft_chain_follows_previous_token(seed):
+    A, Bf = _chain_factors()
+    base, u, anchor = _chain_inputs(seed)
+    d = oracle.draft(base, A, Bf, anchor, u)
+    _check_chain(d, base, anchor)
+    # the chain's tokens are distinct from the first one: biasing every
+    # position by the anchor would be visible
+    assert np.all(d["t"][:, 1:] != d["t"][:, :1])
+
+
+def test_draft_teacher_forcing_follows_the_teacher():
+    """With a teacher path the bias at position i comes from teacher[i-1]
+    (the anchor at i = 1): the oracle's own draw is f(teacher[i-1]) and q_tok
+    is q at the teacher's token."""
+    A, Bf = _chain_factors()
+    base, u, anchor = _chain_inputs(11)
+    rng = np.random.default_rng(12)
+    teacher = rng.integers(0, CV, size=(CB, CK))
+    chain = _expected_chain(anchor)
+    teacher[teacher == chain] = (teacher[teacher == chain] + 1) % CV   # differs from the free chain
+    d = oracle.draft(base, A, Bf, anchor, u, teacher=teacher)
+    prev = np.concatenate([anchor[:, None].astype(np.int64), teacher[:, :-1]], axis=1)
+    want = np.vectorize(_f)(prev)
+    assert np.array_equal(d["t"], want)
+    assert np.array_equal(d["chain"], teacher)
+    for b in range(CB):
+        for i in range(CK):
+            top = want[b, i]
+            if teacher[b, i] == top:
+                continue
+            q_expected = np.exp(float(base[b, i, teacher[b, i]]) - 60.0 - float(base[b, i, top]))
+            assert abs(d["q_tok"][b, i] - q_expected) <= 1e-9 * q_expected
+
+
+def _planted_draft_step(monkeypatch, mistake):
+    real = oracle.draft_step
+    first = {}
+
+    def wrapped(base_i, A64, Bf64, t_prev, u):
+        if mistake == "anchor":
+            first.setdefault("t", np.array(t_prev))
+            t_prev = first["t"]          # never moves past the anchor
+        elif mistake == "no_bias":
+            A64 = np.zeros_like(A64)
+        return real(base_i, A64, Bf64, t_prev, u)
+
+    monkeypatch.setattr(oracle, "draft_step", wrapped)
+
+
+@pytest.mark.parametrize("mistake", ["anchor", "no_bias"])
+def test_chain_pin_detects_planted_mistakes(monkeypatch, mistake):
+    """Plausible mistakes in the chain (every position biased by the anchor;
+    the bias dropped) must fail the chain pin."""
+    A, Bf = _chain_factors()
+    base, u, anchor = _chain_inputs(0)
+    _planted_draft_step(monkeypatch, mistake)
+    d = oracle.draft(base, A, Bf, anchor, u)
+    with pytest.raises(AssertionError):
+        _check_chain(d, base, anchor)
+
+
+# ---------------------------------------------------------------------------
+# Verification with a forced number of acceptances (teacher forcing of the
+# final token). [Tags] "Speculative Decoding", steps 4-5: after the accepted
+# prefix the next token comes from the target row after it (all accepted) or
+# from the adjusted distribution max(0, p - q) at the first rejection. Target
+# row rho holds two tokens d_rho < e_rho with +60 each (p = 1/2 on each); the
+# draft row of the same position puts all its mass on e_rho. Then the
+# residual max(0, p - q) is 1/2 on d_rho alone (final = d_f for a forced
+# count f < L and any uniform), while the bonus (f = L) draws from both halves
+# (u = 0.75 picks e_L).
+FV, FK = 64, 4
+
+
+def _forced_case():
+    rng = np.random.default_rng(21)
+    B = 1
+    d_tok = np.array([3, 10, 17, 24, 31])
+    e_tok = np.array([40, 45, 50, 55, 60])
+    target = rng.normal(0, 2, size=(FK + 1, FV))
+    target[np.arange(FK + 1), d_tok] = 60.0
+    target[np.arange(FK + 1), e_tok] = 60.0
+    z = rng.normal(0, 2, size=(B, FK, FV))
+    z[0, np.arange(FK), e_tok[:FK]] = 60.0
+    lse = scipy.special.logsumexp(z, axis=-1)
+    tokens = np.array([[7, 8, 9, 11]])
+    q_tok = np.exp(np.take_along_axis(z, tokens[..., None], -1)[..., 0] - lse)
+    return target, z, lse, q_tok, tokens, d_tok, e_tok
+
+
+def _check_forced(target, z, lse, q_tok, tokens, d_tok, e_tok):
+    L = np.array([FK])
+    for f in range(FK + 1):
+        v = oracle.verify(target, np.array([0]), z, lse, q_tok, tokens, L,
+                          np.full((1, FK), 0.5, np.float32), np.array([0.75], np.float32),
+                          forced_accepted=np.array([f]))
+        want = e_tok[FK] if f == FK else d_tok[f]
+        assert v["final"][0] == want, (f, v["final"][0], want)
+        assert v["n_out"][0] == f + 1
+        assert np.array_equal(v["out_tokens"][0, :f], tokens[0, :f])
+        assert v["out_tokens"][0, f] == want
+
+
+def test_verify_forced_acceptances_draw_from_the_right_row():
+    _check_forced(*_forced_case())
+
+
+@pytest.mark.parametrize("mistake", ["q_dropped", "q_added", "row_off_by_one"])
+def test_forced_pin_detects_planted_mistakes(monkeypatch, mistake):
+    """Dropping q from the residual, adding it instead of subtracting it, or
+    reading the row after the rejection must fail the forced-acceptance pin."""
+    real = oracle.softmax
+    if mistake == "q_dropped":
+        monkeypatch.setattr(oracle, "softmax", lambda z: real(z) if np.ndim(z) > 1 else np.zeros_like(z))
+    elif mistake == "q_added":
+        # a sign error: the residual weights become max(0, p + q)
+        monkeypatch.setattr(oracle, "softmax", lambda z: real(z) if np.ndim(z) > 1 else -real(z))
+    else:
+        monkeypatch.setattr(oracle, "softmax",
+                            lambda z: real(np.roll(z, -1, axis=0)) if np.ndim(z) > 1 else real(z))
+    with pytest.raises(AssertionError):
+        _check_forced(*_forced_case())
