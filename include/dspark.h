@@ -145,9 +145,10 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
  * (room for DSPARK_STATIC_SCHEDULE_MAX_ITEMS items, about 192 KB), which every
  * GPU that loads the library holds until the process exits. B*K above that
  * limit returns DSPARK_ERR_INVALID_ARG; other argument rules are those of
- * dspark_schedule. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current, so make the first
- * call on each device before any stream capture. All calls share the one
+ * dspark_schedule. Every call looks up the array's device address on the
+ * current device (cudaGetSymbolAddress, which allocates nothing); the first
+ * call on a device may load the library's device code, so make it before any
+ * stream capture. All calls share the one
  * array, and each call fully rewrites what it reads back, so no state carries
  * over between calls; calls that overlap on the GPU (two streams, or two
  * threads) race on the array and must be serialised by the caller.
@@ -157,18 +158,6 @@ dspark_status dspark_schedule_static(const float* conf_logits, const float* temp
                                      const float* profile_ms, int n_prof, int B, int K,
                                      int32_t* verify_len, float* survival, int64_t* row_start,
                                      int32_t* n_tokens, dspark_stream_t stream);
-
-/* Ask the CUDA runtime to set aside up to `bytes` of the current device's L2
- * for persisting accesses (cudaLimitPersistingL2CacheSize, capped at the
- * device's maximum); *granted (if non-NULL) receives the size in effect. The
- * draft kernel reads the Markov factor Bf with an L2 evict-last hint at every
- * position; a set-aside reserves capacity for such lines at the expense of the
- * rest of the L2. It is empty by default, and on B200 the qwen3-sized draft
- * ran slower with one than without (the logits streamed through L2 need the
- * capacity), so the library never requests one itself. The setting belongs to
- * the calling process's CUDA context and ends with it; call once at set-up,
- * outside stream capture. */
-dspark_status dspark_l2_reserve(size_t bytes, size_t* granted);
 
 /* Synchronise `stream`, return the status recorded in the workspace's error
  * word (DSPARK_OK if none) and clear it; *detail (if non-NULL) receives the

@@ -51,8 +51,6 @@ def _load() -> ctypes.CDLL:
     lib.dspark_read_device_error.restype = I
     lib.dspark_schedule_static.argtypes = [P, P, P, I, I, I, P, P, P, P, S]
     lib.dspark_schedule_static.restype = I
-    lib.dspark_l2_reserve.argtypes = [Z, ctypes.POINTER(ctypes.c_size_t)]
-    lib.dspark_l2_reserve.restype = I
     lib.dspark_status_string.argtypes = [I]
     lib.dspark_status_string.restype = ctypes.c_char_p
     return lib
@@ -163,14 +161,6 @@ def dspark_verify(target_logits, row_start, z, lse_q, q_tok, draft_tokens, verif
         _ptr(n_out, "n_out", torch.int32, B), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
         _stream(stream))
     _check("dspark_verify", st)
-
-
-def dspark_l2_reserve(nbytes: int) -> int:
-    """Set aside up to nbytes of L2 for persisting (evict-last) lines in this
-    process's CUDA context; returns the size granted."""
-    got = ctypes.c_size_t(0)
-    _check("dspark_l2_reserve", lib.dspark_l2_reserve(int(nbytes), ctypes.byref(got)))
-    return int(got.value)
 
 
 def dspark_read_device_error(workspace, stream=None) -> tuple[int, int]:

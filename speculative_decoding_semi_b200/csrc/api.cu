@@ -158,19 +158,6 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
   return from_cuda(launch_verify(a, ws + kScratchOffset + schedule_region(B, K), reinterpret_cast<cudaStream_t>(stream)));
 }
 
-dspark_status dspark_l2_reserve(size_t bytes, size_t* granted) {
-  int dev = 0, max_persist = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
-  if (cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, dev) != cudaSuccess)
-    return DSPARK_ERR_CUDA;
-  const size_t want = std::min(bytes, static_cast<size_t>(max_persist));
-  if (cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, want) != cudaSuccess) return DSPARK_ERR_CUDA;
-  size_t now = 0;
-  if (cudaDeviceGetLimit(&now, cudaLimitPersistingL2CacheSize) != cudaSuccess) return DSPARK_ERR_CUDA;
-  if (granted) *granted = now;
-  return DSPARK_OK;
-}
-
 dspark_status dspark_read_device_error(void* workspace, dspark_stream_t stream, uint32_t* detail) {
   if (workspace == nullptr || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

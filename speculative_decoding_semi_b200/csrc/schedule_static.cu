@@ -6,10 +6,8 @@
 // The scratch lives in g_schedule_scratch below: a file-scope __device__
 // array of fixed size, so every GPU that loads libdspark holds it (about
 // 192 KB) until the process exits. Host code cannot use the array's name as
-// a device address; the first call on each device looks the address up with
-// cudaGetSymbolAddress while that device is current and caches it.
-#include <mutex>
-
+// a device address; every call looks the address up with cudaGetSymbolAddress
+// on the current device.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -21,24 +19,13 @@ constexpr size_t kStaticScratchBytes =
 
 static __device__ __align__(256) unsigned char g_schedule_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void* g_scratch_addr[kMaxDevices];
-cudaError_t g_lookup_status[kMaxDevices];
-
-// Device address of g_schedule_scratch on the current device (looked up once
-// per device; the lookup is the only CUDA call this path adds and it allocates
-// nothing).
+// Device address of g_schedule_scratch on the current device. It is looked
+// up on every call (no allocation, and cheap next to the two launches), so a
+// context that was torn down and rebuilt, e.g. after cudaDeviceReset, never
+// sees a stale address, and a failed lookup is not remembered.
 cudaError_t static_scratch(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_once[dev], [dev] {
-    g_lookup_status[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], g_schedule_scratch);
-  });
-  *out = g_scratch_addr[dev];
-  return g_lookup_status[dev];
+  *out = nullptr;
+  return cudaGetSymbolAddress(out, g_schedule_scratch);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -55,6 +42,8 @@ extern "C" dspark_status dspark_schedule_static(const float* conf_logits, const 
   const void* ptrs[] = {conf_logits, temps, profile_ms, verify_len, survival, row_start, n_tokens};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
+  // the largest layout (B*K at the limit) fills the array exactly
+  if (kStaticErrBytes + dspark::schedule_scratch_bytes(B, K) > kStaticScratchBytes) return DSPARK_ERR_INVALID_ARG;
   void* base = nullptr;
   if (static_scratch(&base) != cudaSuccess || base == nullptr) return DSPARK_ERR_CUDA;
   char* scratch = static_cast<char*>(base);

@@ -33,7 +33,10 @@ def _outputs(B, K):
 def test_static_schedule_matches_workspace_schedule_twice():
     from speculative_decoding_semi_b200 import binding
 
-    for key, seed in (("qwen3", 11), (synth.custom(4, B=512, K=16, V=8, n_prof=4096), 12)):
+    # the last case has B*K = 16384, the limit, where the scratch layout fills
+    # the static array exactly
+    for key, seed in (("qwen3", 11), (synth.custom(4, B=512, K=16, V=8, n_prof=4096), 12),
+                      (synth.custom(4, B=512, K=32, V=8, n_prof=512 * 33), 13)):
         d = _inputs(key, seed)
         B, K = d["conf"].shape
         ws = torch.zeros(binding.dspark_workspace_bytes(B, K, 8, 1), dtype=torch.uint8, device="cuda")
