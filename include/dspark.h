@@ -159,6 +159,32 @@ dspark_status dspark_schedule_static(const float* conf_logits, const float* temp
                                      int32_t* verify_len, float* survival, int64_t* row_start,
                                      int32_t* n_tokens, dspark_stream_t stream);
 
+/* Bound, in microseconds, on every device-wide wait of the kernels that use
+ * this workspace (0 restores the default of one second). A wait that runs
+ * out records DSPARK_ERR_TIMEOUT in the workspace's error word; the kernel
+ * then lets its copies in flight land, frees its tensor memory and returns,
+ * leaving its outputs undefined. The setting is kept in the workspace (word 2
+ * of its first 256 bytes) until changed or dspark_workspace_init clears it;
+ * it is written on `stream`, ordered with the calls that follow there. */
+dspark_status dspark_set_wait_budget(void* workspace, uint32_t microseconds, dspark_stream_t stream);
+
+/* Test hook for failure detection without a GPU fault: make CTA `cta` of the
+ * next kernels that use this workspace skip one publish, so that the other
+ * CTAs' bounded waits run out and report DSPARK_ERR_TIMEOUT.
+ *   DSPARK_INJECT_DRAFT_SLICE_SUMS  the draft skips its slice-sum publish at
+ *                                   position 1;
+ *   DSPARK_INJECT_VERIFY_BARRIER    verify skips its arrival at the first
+ *                                   device-wide barrier;
+ *   DSPARK_INJECT_NONE              clears the hook.
+ * Pair it with a short dspark_set_wait_budget. Kept in the workspace (word 3)
+ * until cleared; written on `stream`. */
+typedef enum {
+  DSPARK_INJECT_NONE = 0,
+  DSPARK_INJECT_DRAFT_SLICE_SUMS = 1,
+  DSPARK_INJECT_VERIFY_BARRIER = 2
+} dspark_inject;
+dspark_status dspark_inject_stall(void* workspace, dspark_inject where, uint32_t cta, dspark_stream_t stream);
+
 /* Synchronise `stream`, return the status recorded in the workspace's error
  * word (DSPARK_OK if none) and clear it; *detail (if non-NULL) receives the
  * offending value or the index of the wait that timed out. */

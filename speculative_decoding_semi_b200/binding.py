@@ -51,6 +51,10 @@ def _load() -> ctypes.CDLL:
     lib.dspark_read_device_error.restype = I
     lib.dspark_schedule_static.argtypes = [P, P, P, I, I, I, P, P, P, P, S]
     lib.dspark_schedule_static.restype = I
+    lib.dspark_set_wait_budget.argtypes = [P, ctypes.c_uint32, S]
+    lib.dspark_set_wait_budget.restype = I
+    lib.dspark_inject_stall.argtypes = [P, I, ctypes.c_uint32, S]
+    lib.dspark_inject_stall.restype = I
     lib.dspark_status_string.argtypes = [I]
     lib.dspark_status_string.restype = ctypes.c_char_p
     return lib
@@ -161,6 +165,19 @@ def dspark_verify(target_logits, row_start, z, lse_q, q_tok, draft_tokens, verif
         _ptr(n_out, "n_out", torch.int32, B), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
         _stream(stream))
     _check("dspark_verify", st)
+
+
+DSPARK_INJECT_NONE, DSPARK_INJECT_DRAFT_SLICE_SUMS, DSPARK_INJECT_VERIFY_BARRIER = 0, 1, 2
+
+
+def dspark_set_wait_budget(workspace, microseconds: int, stream=None) -> None:
+    _check("dspark_set_wait_budget", lib.dspark_set_wait_budget(_ptr(workspace, "workspace", torch.uint8),
+                                                                int(microseconds), _stream(stream)))
+
+
+def dspark_inject_stall(workspace, where: int, cta: int = 0, stream=None) -> None:
+    _check("dspark_inject_stall", lib.dspark_inject_stall(_ptr(workspace, "workspace", torch.uint8), int(where),
+                                                          int(cta), _stream(stream)))
 
 
 def dspark_read_device_error(workspace, stream=None) -> tuple[int, int]:

@@ -158,6 +158,23 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
   return from_cuda(launch_verify(a, ws + kScratchOffset + schedule_region(B, K), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+dspark_status dspark_set_wait_budget(void* workspace, uint32_t microseconds, dspark_stream_t stream) {
+  if (workspace == nullptr || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
+  const uint32_t v = microseconds;  // pageable source: staged before the call returns
+  return from_cuda(cudaMemcpyAsync(static_cast<char*>(workspace) + kErrOffset + 2 * sizeof(unsigned), &v,
+                                   sizeof(v), cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_inject_stall(void* workspace, dspark_inject where, uint32_t cta, dspark_stream_t stream) {
+  if (workspace == nullptr || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
+  if (where != DSPARK_INJECT_NONE && where != DSPARK_INJECT_DRAFT_SLICE_SUMS && where != DSPARK_INJECT_VERIFY_BARRIER)
+    return DSPARK_ERR_INVALID_ARG;
+  if (cta >= (1u << 24)) return DSPARK_ERR_INVALID_ARG;
+  const uint32_t v = where == DSPARK_INJECT_NONE ? 0u : ((static_cast<uint32_t>(where) << 24) | cta);
+  return from_cuda(cudaMemcpyAsync(static_cast<char*>(workspace) + kErrOffset + 3 * sizeof(unsigned), &v,
+                                   sizeof(v), cudaMemcpyHostToDevice, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 dspark_status dspark_read_device_error(void* workspace, dspark_stream_t stream, uint32_t* detail) {
   if (workspace == nullptr || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -32,6 +32,9 @@ constexpr size_t kScratchOffset = kSyncOffset + kSyncBytes;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------ error word
+// Words of the workspace's first 256 bytes: [0] status code, [1] detail,
+// [2] wait budget in microseconds (0 = kWaitBudgetNs), [3] stall injection
+// (a test hook: DSPARK_INJECT_* << 24 | CTA index, 0 = none).
 constexpr unsigned kWaitIterLimit = 1u << 26;           // spins before a wait gives up
 constexpr unsigned long long kWaitBudgetNs = 1000000000ull;  // 1 s of device time
 
@@ -41,6 +44,17 @@ __device__ __forceinline__ void set_error(unsigned* err, unsigned code, unsigned
 
 __device__ __forceinline__ unsigned error_code(const unsigned* err) {
   return *reinterpret_cast<const volatile unsigned*>(err);
+}
+
+// Time after which a device-wide wait of a kernel using this workspace gives up.
+__device__ __forceinline__ unsigned long long wait_budget_ns(const unsigned* err) {
+  const unsigned us = *reinterpret_cast<const volatile unsigned*>(err + 2);
+  return us ? static_cast<unsigned long long>(us) * 1000ull : kWaitBudgetNs;
+}
+
+// True when the test hook asks CTA `cta` to skip the publish of kind `kind`.
+__device__ __forceinline__ bool injected_stall(const unsigned* err, unsigned kind, unsigned cta) {
+  return *reinterpret_cast<const volatile unsigned*>(err + 3) == ((kind << 24) | cta);
 }
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
@@ -65,11 +79,12 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 static __device__ __noinline__ bool wait_at_least(const unsigned* ctr, unsigned target, unsigned* err,
                                            unsigned where) {
   const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long budget = wait_budget_ns(err);
   for (unsigned it = 0; it < kWaitIterLimit; ++it) {
     if (ld_acquire_gpu(ctr) >= target) return true;
     if ((it & 31u) == 31u) {
       if (error_code(err) != 0u) return false;
-      if (globaltimer_ns() - t0 > kWaitBudgetNs) break;
+      if (globaltimer_ns() - t0 > budget) break;
     }
     __nanosleep(40);
   }
@@ -301,6 +316,56 @@ __device__ __forceinline__ int scan_rows128(int n, int lane, double R, Load load
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<unsigned>(b) << 16);
+}
+
+// ------------------------------------------------- exponential in fp64
+// 2^(j/16), j = 0..15, for exp_fine; fill with fill_exp_table before use.
+__device__ __forceinline__ void fill_exp_table(double* t16, int tid) {
+  if (tid < 16) t16[tid] = exp2(static_cast<double>(tid) / 16.0);
+}
+
+// e^(zh + zl) in fp64, for an fp32 value zh and a small fp32 correction zl
+// (the rounding error of zh, |zl| <= ulp(zh)). Table-driven, after Tang's
+// method: zh = n ln2/16 + r with n the integer nearest zh 16/ln2, so that
+// e^(zh+zl) = 2^(n>>4) 2^((n&15)/16) e^(r+zl). r is formed with a two-part
+// constant (Cody and Waite): n kC1 is exact since kC1 has 10 significant bits
+// and |n| < 2^14, and the remainder costs one rounding (~1e-9 absolute at
+// |r| ~ 0.02). e^x - 1 for |x| <= 0.022 is its Taylor series to the fifth
+// power (truncation < 2e-13) in fp32, whose rounding moves 1 + p by ~3e-9;
+// the last step is one fp64 FMA by the exact 2^(n>>4) 2^((n&15)/16). The
+// result's relative error is ~5e-9 for |zh| < 30 (against ~1e-7 for an fp32
+// exponential of an fp32-rounded argument). zh < -708 gives 0, zh > 709
+// gives +inf, NaN propagates.
+__device__ __forceinline__ double exp_fine(float zh, float zl, const double* t16) {
+  constexpr float kInvC = 23.083120654223414f;     // 16 / ln 2
+  constexpr float kC1 = 0.0433349609375f;          // 710 * 2^-14
+  constexpr float kC2 = -1.326215250341961e-05f;   // ln2/16 - kC1
+  if (!(zh >= -708.f)) return zh != zh ? static_cast<double>(zh) : 0.0;
+  if (zh > 709.f) return static_cast<double>(INFINITY);
+  // n = zh 16/ln2 rounded to the nearest integer, by adding 1.5 * 2^23 in one
+  // rounding (exact product): the integer lands in the low mantissa bits
+  const float tn = fmaf(zh, kInvC, 12582912.f);
+  const float n = __fsub_rn(tn, 12582912.f);
+  const int ni = __float_as_int(tn) - 0x4B400000;
+  float r = fmaf(-n, kC1, zh);
+  r = fmaf(-n, kC2, r);
+  r = __fadd_rn(r, zl);
+  float q = fmaf(r, 1.f / 120.f, 1.f / 24.f);
+  q = fmaf(q, r, 1.f / 6.f);
+  q = fmaf(q, r, 0.5f);
+  q = fmaf(q, r, 1.f);
+  const float p = __fmul_rn(q, r);
+  const double t = t16[ni & 15];
+  // t is in [1, 2); adding (n >> 4) to its exponent field scales it by
+  // 2^(n>>4), within the normal range for |zh| <= 709
+  const double ts = __hiloint2double(__double2hiint(t) + (ni >> 4) * (1 << 20), __double2loint(t));
+  return fma(ts, static_cast<double>(p), ts);
+}
+
+// fp32 -> bf16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
+  const unsigned u = __float_as_uint(x);
+  return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
 }
 
 }  // namespace dspark

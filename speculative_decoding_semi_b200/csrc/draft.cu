@@ -9,7 +9,8 @@
 // One persistent cooperative kernel runs all K positions. CTA g owns a
 // contiguous vocabulary chunk for every request. Per position i:
 //   1. z = base + A[t_{i-1}] . Bf for the chunk, written to HBM, with the
-//      chunk max m_c and the fp64 sum S_c of exp(z - m_c) per request;
+//      fp64 sum S_c of exp(z) per request (shift 0; the weight carries the
+//      fp32 rounding error of z, found by TwoSum, through exp_fine);
 //   2. device-wide arrival (bounded wait);
 //   3. request b is selected by CTA b mod G: it combines the G chunk partials
 //      in vocabulary order, finds the chunk holding u*W and rescans that chunk
@@ -40,11 +41,12 @@ __device__ __forceinline__ float factor_at(const void* p, long long idx) {
 template <bool BF16>
 __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
   extern __shared__ float arow[];  // [RB][r]
-  __shared__ float redf[32];
   __shared__ double redd[33];
-  __shared__ float s_m[RB];
   __shared__ int s_flag;
   __shared__ int s_tok[RB];
+  __shared__ double t16[16];
+  fill_exp_table(t16, threadIdx.x);
+  __syncthreads();
   const int G = gridDim.x, g = blockIdx.x, tid = threadIdx.x;
   const int NU = a.V / 8;
   const int lo = static_cast<int>(static_cast<long long>(g) * NU / G) * 8;
@@ -62,9 +64,9 @@ __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
         arow[bb * r + k] = factor_at<BF16>(a.A, static_cast<long long>(s_tok[bb]) * r + k);
       }
       __syncthreads();
-      float mx[RB];
+      double S[RB];
 #pragma unroll
-      for (int bb = 0; bb < RB; ++bb) mx[bb] = -INFINITY;
+      for (int bb = 0; bb < RB; ++bb) S[bb] = 0.0;
       for (int v = lo + tid; v < hi; v += DT) {
         float acc[RB];
 #pragma unroll
@@ -78,27 +80,12 @@ __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
         for (int bb = 0; bb < RB; ++bb) {
           if (bb < nb) {
             const long long o = (static_cast<long long>(b0 + bb) * a.K + i) * a.V + v;
-            const float zz = a.base[o] + acc[bb];
+            const float x0 = a.base[o], y0 = acc[bb];
+            const float zz = __fadd_rn(x0, y0);
+            const float yv = __fsub_rn(zz, x0);
+            const float err = __fadd_rn(__fsub_rn(x0, __fsub_rn(zz, yv)), __fsub_rn(y0, yv));
             a.z[o] = zz;
-            mx[bb] = fmaxf(mx[bb], zz);
-          }
-        }
-      }
-#pragma unroll
-      for (int bb = 0; bb < RB; ++bb) {
-        const float m = block_max<DT>(mx[bb], redf);
-        if (tid == 0) s_m[bb] = m;
-      }
-      __syncthreads();
-      double S[RB];
-#pragma unroll
-      for (int bb = 0; bb < RB; ++bb) S[bb] = 0.0;
-      for (int v = lo + tid; v < hi; v += DT) {
-#pragma unroll
-        for (int bb = 0; bb < RB; ++bb) {
-          if (bb < nb) {
-            const long long o = (static_cast<long long>(b0 + bb) * a.K + i) * a.V + v;
-            S[bb] += static_cast<double>(expf(a.z[o] - s_m[bb]));
+            S[bb] += exp_fine(zz, err, t16);
           }
         }
       }
@@ -106,7 +93,7 @@ __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
       for (int bb = 0; bb < RB; ++bb) {
         const double tot = block_sum<DT>(S[bb], redd);
         if (tid == 0 && bb < nb) {
-          a.part_m[static_cast<long long>(b0 + bb) * G + g] = s_m[bb];
+          a.part_m[static_cast<long long>(b0 + bb) * G + g] = 0.f;
           a.part_S[static_cast<long long>(b0 + bb) * G + g] = tot;
         }
       }
@@ -118,7 +105,7 @@ __global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
     if (g < a.B) {
       if (!cta_wait_at_least<CtaSync>(&a.sync[2 * i], static_cast<unsigned>(G), a.err, 2u * i, &s_flag)) return;
       for (int b = g; b < a.B; b += G) {
-        select_token<DT, CtaSync>(a, b, i, G, 8);
+        select_token<DT, CtaSync>(a, b, i, G, 8, t16);
         cta_release_add<CtaSync>(&a.sync[2 * i + 1], 1u);
       }
     }

@@ -27,12 +27,20 @@ __device__ __forceinline__ void chunk_bounds(int V, int unit, int G, int c, int*
   *hi = static_cast<int>(static_cast<long long>(c + 1) * U / G) * unit;
 }
 
-// First element k of z[lo,hi) at which the running sum of exp(z_k - m) * f
-// exceeds R (strict '>'), with each thread scanning a contiguous stretch; if
-// rounding leaves no such element, the last one with a positive weight.
-// Returns the index (>= lo) to every thread.
+// Weight of logit z with shift m and factor f: fp32 exp(z - m) f for a row
+// redrawn with its own maximum (m != 0), fp64 exp(z) f otherwise.
+__device__ __forceinline__ double shifted_weight(float z, float m, double f, const double* t16) {
+  if (m == 0.f) return __dmul_rn(exp_fine(z, 0.f, t16), f);
+  return __dmul_rn(static_cast<double>(expf(z - m)), f);
+}
+
+// First element k of z[lo,hi) at which the running sum of the weights
+// shifted_weight(z_k, m, f) exceeds R (strict '>'), with each thread scanning a
+// contiguous stretch; if rounding leaves no such element, the last one with a
+// positive weight. Returns the index (>= lo) to every thread.
 template <int NT, class Sync>
-__device__ __forceinline__ int rescan_range(const float* zrow, int lo, int hi, float m, double f, double R) {
+__device__ __forceinline__ int rescan_range(const float* zrow, int lo, int hi, float m, double f, double R,
+                                            const double* t16) {
   __shared__ double redd[33];
   __shared__ int redi[32];
   const int tid = threadIdx.x;
@@ -41,7 +49,7 @@ __device__ __forceinline__ int rescan_range(const float* zrow, int lo, int hi, f
   double lw = 0.0;
   int last_pos = -1;
   for (int k = e_lo; k < e_hi; ++k) {
-    const double w = __dmul_rn(static_cast<double>(expf(__ldcg(zrow + k) - m)), f);
+    const double w = shifted_weight(__ldcg(zrow + k), m, f, t16);
     lw += w;
     if (w > 0.0) last_pos = k;
   }
@@ -51,7 +59,7 @@ __device__ __forceinline__ int rescan_range(const float* zrow, int lo, int hi, f
   if (e_lo < e_hi && ex + lw > R) {
     double cum = ex;
     for (int k = e_lo; k < e_hi; ++k) {
-      const double w = __dmul_rn(static_cast<double>(expf(__ldcg(zrow + k) - m)), f);
+      const double w = shifted_weight(__ldcg(zrow + k), m, f, t16);
       cum += w;
       if (cum > R && w > 0.0) {
         found = k;
@@ -69,16 +77,16 @@ __device__ __forceinline__ int rescan_range(const float* zrow, int lo, int hi, f
 // (m_c, S_c = sum_{v in chunk c} exp(z_v - m_c)); chunk c covers the
 // vocabulary slice chunk_bounds(V, unit, G, c). The chunks are combined in
 // vocabulary order in fp64 with the common shift M = max m_c; the chunk whose
-// inclusive prefix first exceeds u*W is rescanned with the same weights
-// exp(z - m_c) * exp(m_c - M) (bit-identical to the ones summed when m_c is
-// the shift used by the producer), and the first element whose running sum
-// exceeds the remainder is the token (strict '>', so a zero weight is never
-// drawn). If W is not a normal positive number (the producer's shift left
-// every weight underflowing or some overflowing), the row is redone with its
-// exact maximum as the shift. Writes draft_tokens, q_tok = w_t / W and
+// inclusive prefix first exceeds u*W is rescanned with the weights
+// exp(z - m_c) * exp(m_c - M) of the stored fp32 z (the producer's sums also
+// carried z's rounding error; the difference is confined to one chunk), and
+// the first element whose running sum exceeds the remainder is the token
+// (strict '>', so a zero weight is never drawn). If W leaves [1e-280, 1e280]
+// (every weight underflowing or some overflowing fp64), the row is redone with
+// its exact maximum as the shift. Writes draft_tokens, q_tok = w_t / W and
 // lse_q = M + log W. All NT threads call.
 template <int NT, class Sync>
-__device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int G, int unit) {
+__device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int G, int unit, const double* t16) {
   __shared__ float redf[32];
   __shared__ double redd[33];
   __shared__ int redi[32];
@@ -104,7 +112,7 @@ __device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int 
   int t;
   float m_t;
   double f_t;
-  if (W >= 1e-30 && W <= 1e30) {
+  if (W >= 1e-280 && W <= 1e280) {
     const double thr = u * W;
     int c = block_min_int<NT, Sync>((tid < G && ex + wc > thr) ? tid : 0x7fffffff, redi);
     if (c == 0x7fffffff) c = G - 1;
@@ -115,14 +123,14 @@ __device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int 
     chunk_bounds(a.V, unit, G, c, &lo, &hi);
     m_t = __ldcg(a.part_m + pb + c);
     f_t = exp(static_cast<double>(m_t) - static_cast<double>(M));
-    t = rescan_range<NT, Sync>(zrow, lo, hi, m_t, f_t, R);
+    t = rescan_range<NT, Sync>(zrow, lo, hi, m_t, f_t, R, t16);
   } else {
     // whole row with its exact maximum as the shift
     float mx = -INFINITY;
     for (int k = tid; k < a.V; k += NT) mx = fmaxf(mx, __ldcg(zrow + k));
     M = block_max<NT, Sync>(mx, redf);
     double s = 0.0;
-    for (int k = tid; k < a.V; k += NT) s += static_cast<double>(expf(__ldcg(zrow + k) - M));
+    for (int k = tid; k < a.V; k += NT) s += shifted_weight(__ldcg(zrow + k), M, 1.0, t16);
     W = block_sum<NT, Sync>(s, redd);
     if (!(W > 0.0) || !(W < INFINITY)) {  // non-finite logits
       if (tid == 0) {
@@ -142,7 +150,7 @@ __device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int 
       const int per = (a.V + NT - 1) / NT;
       const int e_lo = min(a.V, tid * per), e_hi = min(a.V, e_lo + per);
       double lw = 0.0;
-      for (int k = e_lo; k < e_hi; ++k) lw += static_cast<double>(expf(__ldcg(zrow + k) - M));
+      for (int k = e_lo; k < e_hi; ++k) lw += shifted_weight(__ldcg(zrow + k), M, 1.0, t16);
       double tot;
       const double exs = block_exclusive_scan<NT, Sync>(lw, redd, &tot);
       if (e_hi == a.V && e_lo < e_hi) s_W = exs + lw;
@@ -151,10 +159,10 @@ __device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int 
       Sync::sync();
     }
     W = Wscan;
-    t = rescan_range<NT, Sync>(zrow, 0, a.V, M, 1.0, u * W);
+    t = rescan_range<NT, Sync>(zrow, 0, a.V, M, 1.0, u * W, t16);
   }
   if (tid == 0) {
-    const double w_t = __dmul_rn(static_cast<double>(expf(__ldcg(zrow + t) - m_t)), f_t);
+    const double w_t = shifted_weight(__ldcg(zrow + t), m_t, f_t, t16);
     a.tokens[o] = t;
     a.q_tok[o] = static_cast<float>(w_t / W);
     a.lse_q[o] = static_cast<double>(M) + log(W);

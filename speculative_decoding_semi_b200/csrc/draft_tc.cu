@@ -31,10 +31,15 @@
 //              group's tokens before releasing the next position.
 // The epilogue streams base and z through per-warp TMA rings (L2 evict-first)
 // that run ahead across positions, since they do not depend on the tokens.
-// The exponentials use a fixed shift of 0, so each weight is exp(z) itself and
-// every level of the search sums the same fp32 weights in fp64; a row whose
-// sum leaves [1e-30, 1e30] is redone by the selector with its exact maximum.
-// Every wait is bounded and reports DSPARK_ERR_TIMEOUT.
+// Weights. z = base + bias is rounded to fp32 for the output; its rounding
+// error (TwoSum, kept in bf16, ~1e-9 of z) is carried into the weight, which
+// is exp(z) in fp64 (exp_fine, relative error ~5e-9) with a fixed shift of 0,
+// so the sums that place the draw differ from exact ones by ~1e-10 of the row's
+// mass instead of the ~3e-9 an fp32 exponential of the rounded z would give.
+// The last level of the search reads the stored fp32 z; the error there is
+// confined to one 32-row unit. A row whose sum leaves [1e-280, 1e280] is
+// redone by the selector with its exact maximum as the shift. Every wait is
+// bounded and reports DSPARK_ERR_TIMEOUT.
 #include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -50,7 +55,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                   // four per TMEM lane quadrant
 constexpr int kProdWarp = kEpiWarps;
 constexpr int kMmaWarp = kEpiWarps + 1;
 constexpr int kSelWarp = kEpiWarps + 2;
@@ -61,14 +66,18 @@ constexpr int kKStage = 64;                     // r per Bf stage (one 128-byte 
 constexpr int kMaxBfStages = 8;
 constexpr int kBfBoxBytes = 64 * kKStage * 2;   // 64 vocabulary x 64 r, bf16
 constexpr int kBfStageBytes = 2 * kBfBoxBytes;  // a 128-row tile
-constexpr int kChunk = 32;                      // requests per TMEM load and per z box
-constexpr int kBoxBytes = kChunk * kUnit * 4;   // 32 requests x 32 vocabulary, fp32
+constexpr int kChunk = 32;                      // requests per group granule
+constexpr int kSub = 16;                        // requests per TMEM load and per z box
+constexpr int kBoxBytes = kSub * kUnit * 4;     // 16 requests x 32 vocabulary, fp32
 constexpr int kMaxGroup = 128;                  // requests per MMA (N)
 constexpr int kMaxGroups = 4;                   // so B <= 512 on this path
 constexpr int kMaxRingSlots = 8;
 constexpr int kMaxAccSlots = 8;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarBytes = 1024;
+constexpr int kBarBytes = 2048;
+constexpr int kLoBoxBytes = kSub * kUnit * 2;    // bf16 rounding errors of one z box
+constexpr int kSubPerWarp = kMaxGroup / kSub / 4;  // sub-chunks of a group per epilogue warp
+constexpr double kSumLo = 1e-280, kSumHi = 1e280;  // row sums handled with the fixed shift
 
 
 struct TcParams {
@@ -88,7 +97,7 @@ struct TcParams {
 };
 
 struct Layout {
-  int bf, brows, ring, part, bar, misc, total;
+  int bf, brows, ring, lo, part, bar, tab, misc, total;
 };
 
 __host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs, int part_bytes) {
@@ -96,57 +105,43 @@ __host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs,
   L.bf = 0;
   L.brows = L.bf + nbf * kBfStageBytes;
   L.ring = L.brows + ((brows_bytes + 1023) / 1024) * 1024;
-  L.part = L.ring + kEpiWarps * nbs * kBoxBytes;
+  L.lo = L.ring + kEpiWarps * nbs * kBoxBytes;
+  L.part = L.lo + kEpiWarps * kLoBoxBytes;
   L.bar = L.part + ((part_bytes + 15) / 16) * 16;
-  L.misc = L.bar + kBarBytes;
+  L.tab = L.bar + kBarBytes;
+  L.misc = L.tab + 16 * 8;
   L.total = L.misc + 64;
   return L;
 }
 
+// The kernel's mbarriers, addressed from one base pointer (one register
+// rather than one per array).
 struct Bars {
-  uint64_t* bf_full;       // [kMaxBfStages]
-  uint64_t* bf_empty;      // [kMaxBfStages]
-  uint64_t* acc_full;      // [kMaxAccSlots]
-  uint64_t* acc_empty;     // [kMaxAccSlots]
-  uint64_t* brows_full;
-  uint64_t* mma_done;
-  uint64_t* final_mma;
-  uint64_t* tokens_ready;  // [kMaxGroups]
-  uint64_t* step_done;     // [kMaxGroups]
-  uint64_t* base_full;     // [kEpiWarps][kMaxRingSlots]
+  uint64_t* q;
+  __device__ uint64_t* bf_full(int s) const { return q + s; }
+  __device__ uint64_t* bf_empty(int s) const { return q + kMaxBfStages + s; }
+  __device__ uint64_t* acc_full(int s) const { return q + 2 * kMaxBfStages + s; }
+  __device__ uint64_t* acc_empty(int s) const { return q + 2 * kMaxBfStages + kMaxAccSlots + s; }
+  __device__ uint64_t* brows_full() const { return q + 2 * kMaxBfStages + 2 * kMaxAccSlots; }
+  __device__ uint64_t* mma_done() const { return brows_full() + 1; }
+  __device__ uint64_t* final_mma() const { return brows_full() + 2; }
+  __device__ uint64_t* tokens_ready(int g) const { return brows_full() + 3 + g; }
+  __device__ uint64_t* step_done(int g) const { return brows_full() + 3 + kMaxGroups + g; }
+  __device__ uint64_t* base_full(int s) const { return brows_full() + 3 + 2 * kMaxGroups + s; }
 };
 
-__device__ __forceinline__ Bars carve_bars(uint8_t* p) {
-  Bars b;
-  uint64_t* q = reinterpret_cast<uint64_t*>(p);
-  b.bf_full = q;
-  q += kMaxBfStages;
-  b.bf_empty = q;
-  q += kMaxBfStages;
-  b.acc_full = q;
-  q += kMaxAccSlots;
-  b.acc_empty = q;
-  q += kMaxAccSlots;
-  b.brows_full = q++;
-  b.mma_done = q++;
-  b.final_mma = q++;
-  b.tokens_ready = q;
-  q += kMaxGroups;
-  b.step_done = q;
-  q += kMaxGroups;
-  b.base_full = q;
-  return b;
-}
+__device__ __forceinline__ Bars carve_bars(uint8_t* p) { return Bars{reinterpret_cast<uint64_t*>(p)}; }
 
 __device__ __forceinline__ int group_real(const TcParams& p, int gr) { return min(p.gsize, p.d.B - gr * p.gsize); }
 __device__ __forceinline__ int round16(int n) { return (n + 15) & ~15; }
-// Epilogue half h takes chunks c (32 requests each) with c % 2 == h ^ (gr % 2)
-// of group gr: with one chunk per group the two halves take alternate groups.
-__device__ __forceinline__ int half_of(int h, int gr) { return h ^ (gr & 1); }
-// chunks c with c % 2 == hh among the group's real columns
+// Epilogue warp h of a quadrant (0..3) takes the group's sub-chunks s (16
+// requests each) with s % 4 == (h + gr) % 4: the rotation spreads groups whose
+// sub-chunk count is not a multiple of 4 over all four warps.
+__device__ __forceinline__ int half_of(int h, int gr) { return (h + gr) & 3; }
+// sub-chunks s with s % 4 == hh among the group's real columns
 __device__ __forceinline__ int chunks_for(int ncol, int hh) {
-  const int nch = (ncol + kChunk - 1) / kChunk;
-  return nch > hh ? (nch - hh + 1) / 2 : 0;
+  const int nsub = (ncol + kSub - 1) / kSub;
+  return nsub > hh ? (nsub - hh + 3) / 4 : 0;
 }
 
 // Tile visited t-th in pass (i, gr): passes over the slice alternate
@@ -295,8 +290,6 @@ __device__ __forceinline__ int warp_search(int n, Get get, Thr thr_of, int lane,
   return best;
 }
 
-// exp(z): the weight of the epilogue's slice sums and of the selector's rescan.
-__device__ __forceinline__ float zw(float z) { return expf(z); }
 
 // Draw from the whole row z with its exact maximum as the shift, for a row
 // whose sum of exp(z) leaves [1e-30, 1e30] (one warp). Non-finite logits are
@@ -323,11 +316,11 @@ __device__ __noinline__ int draw_full_row(const float* zrow, int V, double u, in
 }
 
 // Draw request b's token at position i (one warp) by a three-level
-// inverse-CDF search over the same fp64 sums of the weights exp(z): the G
-// slice sums (whose total is the W that u scales), the chosen slice's sums over
-// its 32-row units, then the chosen unit's 32 weights. Writes draft_tokens,
-// q_tok and lse_q; returns the token.
-__device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane) {
+// inverse-CDF search over fp64 sums of the weights exp(z): the G slice sums
+// (whose total is the W that u scales), the chosen slice's sums over its 32-row
+// units, then the chosen unit's 32 weights (from the stored fp32 z). Writes
+// draft_tokens, q_tok and lse_q; returns the token.
+__device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane, const double* t16) {
   const DraftArgs& d = p.d;
   const long long o = static_cast<long long>(b) * d.K + i;
   const float* zrow = d.z + o * d.V;
@@ -337,11 +330,11 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
   // level 1: slice sums; their total is the W that u scales
   const int c = warp_search<8>(
       G, [&](int cc) { return __ldcg(part + cc); },
-      [&](double tot) { return (tot >= 1e-30 && tot <= 1e30) ? u * tot : INFINITY; }, lane, &ex, &W);
+      [&](double tot) { return (tot >= kSumLo && tot <= kSumHi) ? u * tot : INFINITY; }, lane, &ex, &W);
   int tok;
   double w_t;
   float shift = 0.f;
-  if (W >= 1e-30 && W <= 1e30) {
+  if (W >= kSumLo && W <= kSumHi) {
     const double R = u * W - ex;
     // level 2: the slice's unit sums, in vocabulary order
     int lo, hi;
@@ -354,7 +347,7 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
                              [&](double) { return R; }, lane, &ex2, &tot2);
     const double R2 = R - ex2;
     // level 3: the unit's weights, one per lane
-    const double w = static_cast<double>(zw(__ldcg(zrow + static_cast<long long>(ux) * kUnit + lane)));
+    const double w = exp_fine(__ldcg(zrow + static_cast<long long>(ux) * kUnit + lane), 0.f, t16);
     const double inc = warp_inclusive_scan(w);
     const unsigned hit = __ballot_sync(0xffffffffu, inc > R2 && w > 0.0);
     const unsigned pos = __ballot_sync(0xffffffffu, w > 0.0);
@@ -398,7 +391,8 @@ __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned 
   return ok;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// 19 warps: five share a 16K-register SM sub-partition, so at most 96 registers each
+__global__ void __maxnreg__(96)
     draft_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_bf,
                     const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_z) {
   extern __shared__ uint8_t smem_raw[];
@@ -409,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
   double* s_part = reinterpret_cast<double*>(smem + Ly.part);  // [group][quadrant][gsize]
+  double* t16 = reinterpret_cast<double*>(smem + Ly.tab);      // 2^(j/16) for exp_fine
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = gridDim.x, g = blockIdx.x;
@@ -419,24 +414,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kMaxBfStages; ++s) {
-      mbar_init(&bars.bf_full[s], 1);
-      mbar_init(&bars.bf_empty[s], 1);
+      mbar_init(bars.bf_full(s), 1);
+      mbar_init(bars.bf_empty(s), 1);
     }
     for (int s = 0; s < kMaxAccSlots; ++s) {
-      mbar_init(&bars.acc_full[s], 1);
-      mbar_init(&bars.acc_empty[s], kEpiWarps);
+      mbar_init(bars.acc_full(s), 1);
+      mbar_init(bars.acc_empty(s), kEpiWarps);
     }
-    mbar_init(bars.brows_full, 1);
-    mbar_init(bars.mma_done, 1);
-    mbar_init(bars.final_mma, 1);
+    mbar_init(bars.brows_full(), 1);
+    mbar_init(bars.mma_done(), 1);
+    mbar_init(bars.final_mma(), 1);
     for (int s = 0; s < kMaxGroups; ++s) {
-      mbar_init(&bars.tokens_ready[s], 1);
-      mbar_init(&bars.step_done[s], kEpiWarps);
+      mbar_init(bars.tokens_ready(s), 1);
+      mbar_init(bars.step_done(s), kEpiWarps);
     }
-    for (int s = 0; s < kEpiWarps * kMaxRingSlots; ++s) mbar_init(&bars.base_full[s], 1);
+    for (int s = 0; s < kEpiWarps * kMaxRingSlots; ++s) mbar_init(bars.base_full(s), 1);
     *s_abort = 0;
     fence_mbar_init();
   }
+  fill_exp_table(t16, threadIdx.x);
   if (warp == kMmaWarp) {
     tmem_alloc(s_tmem, kTmemCols);
     tmem_relinquish();
@@ -461,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int gr = 0; ok && gr < p.ngroups; ++gr)
           for (int t = 0; ok && t < ntiles; ++t)
             for (int s = 0; s < p.r_stages; ++s) {
-              if (!mbar_wait(&bars.bf_empty[stage], phase ^ 1u, s_abort, d.err, 0x100u)) {
+              if (!mbar_wait(bars.bf_empty(stage), phase ^ 1u, s_abort, d.err, 0x100u)) {
                 ok = false;
                 break;
               }
@@ -471,9 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               // a last tile of at most 64 rows needs only the first 64-row box:
               // the MMA's rows beyond it are never read by the epilogue
               const bool both = (pt == ntiles - 1 ? last_rows : kTileRows) > 64;
-              mbar_arrive_expect_tx(&bars.bf_full[stage], both ? kBfStageBytes : kBfBoxBytes);
-              tma_load_2d(dst, &tm_bf, v0, s * kKStage, &bars.bf_full[stage], pol);
-              if (both) tma_load_2d(dst + kBfBoxBytes, &tm_bf, v0 + 64, s * kKStage, &bars.bf_full[stage], pol);
+              mbar_arrive_expect_tx(bars.bf_full(stage), both ? kBfStageBytes : kBfBoxBytes);
+              tma_load_2d(dst, &tm_bf, v0, s * kKStage, bars.bf_full(stage), pol);
+              if (both) tma_load_2d(dst + kBfBoxBytes, &tm_bf, v0 + 64, s * kKStage, bars.bf_full(stage), pol);
               issued[stage] = true;
               issued_parity[stage] = phase;
               if (++stage == p.nbf) {
@@ -483,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
       // every load lands before the CTA can exit
       for (int s = 0; s < p.nbf; ++s)
-        if (issued[s]) mbar_drain(&bars.bf_full[s], issued_parity[s], d.err, 0x101u);
+        if (issued[s]) mbar_drain(bars.bf_full(s), issued_parity[s], d.err, 0x101u);
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA
@@ -501,24 +497,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t idesc = idesc_bf16_f32(N, 1);
           // the operand buffer is free once the previous group's MMAs are done
           if (brows_used) {
-            mma_commit(bars.mma_done);
-            if (!mbar_wait(bars.mma_done, done_phase, s_abort, d.err, 0x204u)) {
+            mma_commit(bars.mma_done());
+            if (!mbar_wait(bars.mma_done(), done_phase, s_abort, d.err, 0x204u)) {
               ok = false;
               break;
             }
             done_phase ^= 1u;
           }
-          if (!mbar_wait(&bars.tokens_ready[gr], tr_phase[gr], s_abort, d.err, 0x200u)) {
+          if (!mbar_wait(bars.tokens_ready(gr), tr_phase[gr], s_abort, d.err, 0x200u)) {
             ok = false;
             break;
           }
           tr_phase[gr] ^= 1u;
           fence_proxy_async_all();
           const uint32_t bytes = static_cast<uint32_t>(N * d.r * 2);
-          mbar_arrive_expect_tx(bars.brows_full, bytes);
+          mbar_arrive_expect_tx(bars.brows_full(), bytes);
           bulk_load(smem + Ly.brows, p.image + static_cast<long long>(gr) * p.image_stride, bytes,
-                    bars.brows_full);
-          if (!mbar_wait(bars.brows_full, brows_phase, s_abort, d.err, 0x205u)) {
+                    bars.brows_full());
+          if (!mbar_wait(bars.brows_full(), brows_phase, s_abort, d.err, 0x205u)) {
             ok = false;
             break;
           }
@@ -526,14 +522,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           brows_used = true;
           tc_fence_after();
           for (int t = 0; ok && t < ntiles; ++t) {
-            if (!mbar_wait(&bars.acc_empty[slot], slot_phase ^ 1u, s_abort, d.err, 0x201u)) {
+            if (!mbar_wait(bars.acc_empty(slot), slot_phase ^ 1u, s_abort, d.err, 0x201u)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t dcol = tmem_base + static_cast<uint32_t>(slot * p.slot_stride);
             for (int s = 0; s < p.r_stages; ++s) {
-              if (!mbar_wait(&bars.bf_full[stage], phase, s_abort, d.err, 0x202u)) {
+              if (!mbar_wait(bars.bf_full(stage), phase, s_abort, d.err, 0x202u)) {
                 ok = false;
                 break;
               }
@@ -546,14 +542,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t bdesc = smem_desc_sw128(b_base + kk * 32, 16, 1024);
                 mma_bf16(dcol, adesc, bdesc, idesc, (s | kk) != 0);
               }
-              mma_commit(&bars.bf_empty[stage]);
+              mma_commit(bars.bf_empty(stage));
               if (++stage == p.nbf) {
                 stage = 0;
                 phase ^= 1u;
               }
             }
             if (!ok) break;
-            mma_commit(&bars.acc_full[slot]);
+            mma_commit(bars.acc_full(slot));
             if (++slot == p.nslots) {
               slot = 0;
               slot_phase ^= 1u;
@@ -561,8 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       // all issued MMAs complete before TMEM is released
-      mma_commit(bars.final_mma);
-      mbar_drain(bars.final_mma, 0, d.err, 0x203u);
+      mma_commit(bars.final_mma());
+      mbar_drain(bars.final_mma(), 0, d.err, 0x203u);
     }
   } else if (warp == kSelWarp) {
     // ------------------------------------------------------------ selector
@@ -594,12 +590,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int gr = 0; ok && gr < p.ngroups; ++gr) {
       ok = warp_wait_counter(&p.sync_tok[gr], static_cast<unsigned>(group_real(p, gr)), d.err, 0x400u + gr,
                              s_abort, lane);
-      if (ok && lane == 0) mbar_arrive(&bars.tokens_ready[gr]);
+      if (ok && lane == 0) mbar_arrive(bars.tokens_ready(gr));
     }
     for (int i = 0; ok && i < d.K; ++i) {
       for (int gr = 0; ok && gr < p.ngroups; ++gr) {
         const int gbase = gr * p.gsize, nreal = group_real(p, gr);
-        if (!mbar_wait(&bars.step_done[gr], i & 1, s_abort, d.err, 0x500u)) {
+        if (!mbar_wait(bars.step_done(gr), i & 1, s_abort, d.err, 0x500u)) {
           ok = false;
           break;
         }
@@ -612,7 +608,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         const unsigned slot = static_cast<unsigned>(i * p.ngroups + gr);
-        if (lane == 0) red_release_gpu_add(&p.sync_part[slot], 1u);
+        // (test hook: one CTA may skip its publish at position 1 so that the
+        // other CTAs' waits run out)
+        if (lane == 0 && !(i == 0 && injected_stall(d.err, DSPARK_INJECT_DRAFT_SLICE_SUMS, g)))
+          red_release_gpu_add(&p.sync_part[slot], 1u);
         unsigned mine = 0;
         // first request of this group drawn by CTA g: the smallest b >= gbase with b % G == g
         const int first = gbase + ((g - gbase) % G + G) % G;
@@ -620,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = warp_wait_counter(&p.sync_part[slot], static_cast<unsigned>(G), d.err, 0x600u + slot, s_abort, lane);
           if (!ok) break;
           for (int b = first; b < gbase + nreal; b += G) {
-            const int t = select_warp(p, b, i, G, lane);
+            const int t = select_warp(p, b, i, G, lane, t16);
             if (i + 1 < d.K) write_image_row(p, b, t, lane);
             ++mine;
           }
@@ -631,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0 && mine) red_release_gpu_add(&p.sync_tok[nslot], mine);
           ok = warp_wait_counter(&p.sync_tok[nslot], static_cast<unsigned>(nreal), d.err, 0x700u + nslot, s_abort,
                                  lane);
-          if (ok && lane == 0) mbar_arrive(&bars.tokens_ready[gr]);
+          if (ok && lane == 0) mbar_arrive(bars.tokens_ready(gr));
         }
       }
     }
@@ -645,7 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_z);
     }
     float* ring = reinterpret_cast<float*>(smem + Ly.ring + warp * p.nbs * kBoxBytes);
-    uint64_t* rfull = bars.base_full + warp * kMaxRingSlots;
+    uint16_t* lobox = reinterpret_cast<uint16_t*>(smem + Ly.lo + warp * kLoBoxBytes);
+    uint64_t* rfull = bars.base_full(warp * kMaxRingSlots);
     Items L;
     L.p = &p;
     L.ntiles = ntiles;
@@ -658,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = nl % p.nbs;
       mbar_arrive_expect_tx(&rfull[j], kBoxBytes);
       tma_load_3d(ring + j * (kBoxBytes / 4), &tm_base, lo + L.ptile() * kTileRows + kUnit * q, L.i,
-                  L.gr * p.gsize + (2 * L.k + half_of(h, L.gr)) * kChunk, &rfull[j], pol_first);
+                  L.gr * p.gsize + (4 * L.k + half_of(h, L.gr)) * kSub, &rfull[j], pol_first);
       L.next();
       ++nl;
     };
@@ -685,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // hand them, with the lanes' unit sums, to the selector, whose gpu-scope
       // release reduction publishes them
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.step_done[pending]);
+      if (lane == 0) mbar_arrive(bars.step_done(pending));
       pending = -1;
     };
 
@@ -698,36 +698,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nreal = group_real(p, gr);
         const int hh = half_of(h, gr);
         const int nk = chunks_for(nreal, hh);
-        // lane l sums column (request) col0 + l of each chunk over the slice
-        double acc[kMaxGroup / kChunk / 2];
+        // lane l < 16 sums column (request) col0 + l of each sub-chunk over the slice
+        double acc[kSubPerWarp];
 #pragma unroll
-        for (int k = 0; k < kMaxGroup / kChunk / 2; ++k) acc[k] = 0.0;
+        for (int k = 0; k < kSubPerWarp; ++k) acc[k] = 0.0;
         // no stores of this warp follow in this group: release the last one now
         if (nk == 0) release_pending(0);
         for (int t = 0; ok && t < ntiles; ++t) {
           const int pt = phys_tile(i, gr, p.ngroups, ntiles, t);
           const int rows = (pt == ntiles - 1) ? last_rows : kTileRows;
-          ok = mbar_wait(&bars.acc_full[slot], slot_phase, s_abort, d.err, 0x300u);
+          ok = mbar_wait(bars.acc_full(slot), slot_phase, s_abort, d.err, 0x300u);
           if (!ok) break;
           tc_fence_after();
           if (kUnit * q < rows) {
             const int v0 = lo + pt * kTileRows + kUnit * q;
 #pragma unroll
-            for (int kk = 0; kk < kMaxGroup / kChunk / 2; ++kk) {
+            for (int kk = 0; kk < kSubPerWarp; ++kk) {
               if (kk < nk && ok) {
                 const int j = nc % p.nbs;
                 ok = mbar_wait(&rfull[j], (nc / p.nbs) & 1, s_abort, d.err, 0x301u);
                 if (ok) {
                   float* box = ring + j * (kBoxBytes / 4);
-                  const int col0 = (2 * kk + hh) * kChunk;
-                  uint32_t rg[32];
-                  tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(kUnit * q) << 16) +
+                  const int col0 = (4 * kk + hh) * kSub;
+                  uint32_t rg[kSub];
+                  tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(kUnit * q) << 16) +
                                          static_cast<uint32_t>(slot * p.slot_stride + col0),
                                      rg);
                   tmem_ld_wait();
-                  // z = base + bias in place (lane = vocabulary row, c = request)
+                  // z = base + bias in place (lane = vocabulary row, c = request),
+                  // its rounding error by TwoSum into the bf16 box (its upper
+                  // 16 bits: ~2^-8 of an error that is itself below ulp(z));
+                  // the previous sub-chunk's reads of that box are done first
+                  __syncwarp();
 #pragma unroll
-                  for (int c = 0; c < kChunk; ++c) box[c * kUnit + lane] += __uint_as_float(rg[c]);
+                  for (int c = 0; c < kSub; ++c) {
+                    const float x0 = box[c * kUnit + lane], y0 = __uint_as_float(rg[c]);
+                    const float sum = __fadd_rn(x0, y0);
+                    const float yv = __fsub_rn(sum, x0);
+                    const float err = __fadd_rn(__fsub_rn(x0, __fsub_rn(sum, yv)), __fsub_rn(y0, yv));
+                    box[c * kUnit + lane] = sum;
+                    lobox[c * kUnit + lane] = static_cast<uint16_t>(__float_as_uint(err) >> 16);
+                  }
                   fence_proxy_async_shared();
                   __syncwarp();
                   ++nc;
@@ -735,15 +746,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_store_3d(&tm_z, box, v0, i, gbase + col0, pol_first);
                     bulk_commit();
                   }
-                  // the box's sum over its 32 rows for request col0 + lane,
-                  // read across the rows starting at row `lane` so that the
-                  // 32 lanes read 32 different banks
-                  const float* colp = box + lane * kUnit;
-                  double us = 0.0;
-#pragma unroll
-                  for (int k = 0; k < kUnit; ++k) us += static_cast<double>(zw(colp[(k + lane) & (kUnit - 1)]));
-                  const int col = gbase + col0 + lane;
-                  if (col0 + lane < nreal) {
+                  // the box's sum over its 32 rows for request col0 + (lane & 15):
+                  // lane l reads rows 16 (l >> 4) .. + 15, starting at a row
+                  // rotated by the request so that the 32 lanes hit 32 banks;
+                  // the two halves meet in one shuffle
+                  const int cr = lane & (kSub - 1);
+                  const float* colp = box + cr * kUnit + (lane >> 4) * 16;
+                  const uint16_t* lop = lobox + cr * kUnit + (lane >> 4) * 16;
+                  double us0 = 0.0, us1 = 0.0;
+#pragma unroll 4
+                  for (int k = 0; k < 16; k += 2) {
+                    const int k0 = (k + cr) & 15, k1 = (k + 1 + cr) & 15;
+                    us0 += exp_fine(colp[k0], bf16_bits_to_float(lop[k0]), t16);
+                    us1 += exp_fine(colp[k1], bf16_bits_to_float(lop[k1]), t16);
+                  }
+                  double us = us0 + us1;
+                  us += __shfl_xor_sync(0xffffffffu, us, 16);
+                  const int col = gbase + col0 + cr;
+                  if (lane < kSub && col0 + cr < nreal) {
                     acc[kk] += us;
                     p.unit_sum[static_cast<long long>(v0 / kUnit) * d.B + col] = us;
                   }
@@ -757,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.acc_empty[slot]);
+          if (lane == 0) mbar_arrive(bars.acc_empty(slot));
           if (++slot == p.nslots) {
             slot = 0;
             slot_phase ^= 1u;
@@ -767,9 +787,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         // this warp's quadrant of the slice sums of group gr
 #pragma unroll
-        for (int kk = 0; kk < kMaxGroup / kChunk / 2; ++kk) {
-          const int col = (2 * kk + hh) * kChunk + lane;
-          if (kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[kk];
+        for (int kk = 0; kk < kSubPerWarp; ++kk) {
+          const int col = (4 * kk + hh) * kSub + lane;
+          if (lane < kSub && kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[kk];
         }
         release_pending(0);
         pending = gr;
@@ -885,7 +905,7 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.V), static_cast<cuuint64_t>(a.K),
                           static_cast<cuuint64_t>(a.B)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.V) * 4, static_cast<cuuint64_t>(a.V) * a.K * 4};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(kUnit), 1, static_cast<cuuint32_t>(kChunk)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(kUnit), 1, static_cast<cuuint32_t>(kSub)};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,

@@ -56,22 +56,29 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase of `parity` to complete. Gives up if *abort is
-// set by another warp, or after kWaitIterLimit polls / 2*kWaitBudgetNs, in
+// set by another warp, or after kWaitIterLimit polls / twice the wait budget, in
 // which case it records DSPARK_ERR_TIMEOUT (detail `where`) and sets *abort.
-static __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err,
-                                              unsigned where) {
-  if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                   unsigned* err, unsigned where) {
   const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long budget = 2 * wait_budget_ns(err);
   for (unsigned it = 0; it < kWaitIterLimit; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 15u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > 2 * kWaitBudgetNs) break;
+      if (globaltimer_ns() - t0 > budget) break;
     }
   }
   set_error(err, DSPARK_ERR_TIMEOUT, where);
   *abort = 1;
   return false;
+}
+
+// The first test is inline; only a wait that has to spin calls out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err,
+                                          unsigned where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, err, where);
 }
 
 // Wait for copies or MMAs this thread started to finish before the CTA exits

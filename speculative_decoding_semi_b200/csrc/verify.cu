@@ -655,7 +655,10 @@ __device__ bool grid_barrier(const Params& P, int k, int* s_flag) {
   // later reads; separate gpu fences would only add microseconds.
   __syncthreads();
   if (threadIdx.x == 0) {
-    red_release_gpu_add(P.w.ctl + kCtlBar + k, 1u);
+    // (test hook: one CTA may skip its arrival at the first barrier so that
+    // every CTA's wait runs out)
+    if (!(k == 0 && injected_stall(P.a.err, DSPARK_INJECT_VERIFY_BARRIER, blockIdx.x)))
+      red_release_gpu_add(P.w.ctl + kCtlBar + k, 1u);
     const bool ok = wait_at_least(P.w.ctl + kCtlBar + k, gridDim.x, P.a.err, 0x500u + k);
     *s_flag = ok ? 1 : 0;
   }

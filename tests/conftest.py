@@ -25,3 +25,19 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Pooled excused-mismatch counts of the GPU parity tests run here."""
+    mod = sys.modules.get("tests.parity")
+    if mod is None or not getattr(mod, "SUMMARY", None):
+        return
+    terminalreporter.section("parity: excused mismatches (oracle margin < 1e-5) per test")
+    tot_d = tot_e = 0
+    for name, t in mod.SUMMARY.items():
+        tot_d += t["decisions"]
+        tot_e += t["excused"]
+        kinds = ", ".join(f"{k} {v[1]}/{v[0]}" for k, v in sorted(t["by_kind"].items()))
+        terminalreporter.write_line(f"{name}: {t['excused']}/{t['decisions']} "
+                                    f"({100.0 * t['excused'] / max(1, t['decisions']):.4f}%); {kinds}")
+    terminalreporter.write_line(f"all: {tot_e}/{tot_d} ({100.0 * tot_e / max(1, tot_d):.4f}%)")

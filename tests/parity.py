@@ -4,8 +4,8 @@ Integer outputs must match exactly, except where the oracle's own decision
 margin is below MARGIN (1e-5): inverse-CDF margin d < 1e-5, accept margin
 |u - p/q| < 1e-5, or a scheduler near-tie (|P_(m*) - P_(m*+1)| < 1e-5 P_(m*)
 or a runner-up objective within 1e-5). Such mismatches are counted as
-excused and their pooled rate must stay under 0.1% of decisions; any other
-mismatch fails. After an excused mismatch the oracle continues from the GPU's
+excused and their pooled count must stay at or under 0.1% of the decisions
+(a point rate, no allowance for sampling noise); any other mismatch fails. After an excused mismatch the oracle continues from the GPU's
 choice (teacher forcing), so one near-tie counts once.
 Float outputs: q_tok and survival within 2e-3 relative, lse_q within 2e-3
 absolute; z within 1e-4 absolute + 1e-5 relative (fp32 rounding of base +
@@ -14,7 +14,6 @@ bias, with the bias accumulated in fp32).
 from __future__ import annotations
 
 import dataclasses
-import math
 
 import numpy as np
 import torch
@@ -25,6 +24,9 @@ import synth
 MARGIN = 1e-5
 RATE = 1e-3
 
+# Pooled tallies of this process, by test, for the end-of-run summary.
+SUMMARY: dict = {}
+
 
 @dataclasses.dataclass
 class Tally:
@@ -32,33 +34,37 @@ class Tally:
     excused: int = 0
     flagged: int = 0
     failures: list = dataclasses.field(default_factory=list)
+    by_kind: dict = dataclasses.field(default_factory=dict)
 
     def add(self, other: "Tally"):
         self.decisions += other.decisions
         self.excused += other.excused
         self.flagged += other.flagged
         self.failures += other.failures
+        for k, v in other.by_kind.items():
+            a = self.by_kind.setdefault(k, [0, 0])
+            a[0] += v[0]
+            a[1] += v[1]
 
-    def check(self):
+    def count(self, kind: str, decisions: int, excused: int):
+        self.decisions += decisions
+        self.excused += excused
+        a = self.by_kind.setdefault(kind, [0, 0])
+        a[0] += decisions
+        a[1] += excused
+
+    def check(self, name: str | None = None):
+        if name is not None:
+            SUMMARY[name] = {"decisions": self.decisions, "excused": self.excused, "flagged": self.flagged,
+                             "by_kind": {k: list(v) for k, v in self.by_kind.items()}}
         assert not self.failures, self.failures[:10]
-        assert self.excused < excused_limit(self.decisions), (self.excused, self.decisions, self.flagged)
+        assert within_rate(self.excused, self.decisions), (self.excused, self.decisions, self.flagged)
 
 
-def excused_limit(decisions: int, level: float = 0.05) -> int:
-    """Excused mismatches must stay under RATE (0.1%) of the decisions. The
-    count from a finite sample is a Poisson draw, so the check fails when it
-    is significantly above that rate: it returns the smallest k with
-    P(X >= k) < level for X ~ Poisson(RATE * decisions), and at least 2 (one
-    excused near-tie is always allowed). A true rate at the limit then fails
-    5% of samples rather than a third of them at ~1,000 decisions, while a
-    rate ten times higher (fp32 accumulation of the weights) still fails."""
-    lam = RATE * decisions
-    k, term, below = 0, math.exp(-lam), 0.0
-    while 1.0 - below >= level:
-        below += term
-        k += 1
-        term *= lam / k
-    return max(k, 2)
+def within_rate(excused: int, decisions: int) -> bool:
+    """Excused mismatches must stay under RATE (0.1%) of the decisions, as a
+    point rate: excused <= 0.001 * decisions (so none at all below 1,000)."""
+    return excused <= RATE * decisions
 
 
 def compare_draft(inp, gpu, requests, tally: Tally, check_z=True):
@@ -68,9 +74,8 @@ def compare_draft(inp, gpu, requests, tally: Tally, check_z=True):
                      teacher=gpu["tokens"].astype(np.int64), keep_z=True)
     mism = d["t"] != gpu["tokens"]
     small = d["margin"] < MARGIN
-    tally.decisions += mism.size
     tally.flagged += int(small.sum())
-    tally.excused += int((mism & small).sum())
+    tally.count("draft", mism.size, int((mism & small).sum()))
     bad = np.argwhere(mism & ~small)
     for b, i in bad[:5]:
         tally.failures.append(("draft token", int(requests[b]), int(i), int(d["t"][b, i]), int(gpu["tokens"][b, i]),
@@ -96,14 +101,15 @@ def compare_schedule(inp, gpu, tally: Tally):
     if rel.max() > 2e-3:
         tally.failures.append(("survival rel", float(rel.max())))
     B = P.shape[0]
-    tally.decisions += B
     L = gpu["verify_len"]
+    exc = 0
     if not np.array_equal(L, s["verify_len"]):
         if s["gap_item"] < MARGIN or s["gap_obj"] < MARGIN:
-            tally.excused += int((L != s["verify_len"]).sum())
+            exc = int((L != s["verify_len"]).sum())
         else:
             tally.failures.append(("verify_len", np.argwhere(L != s["verify_len"]).ravel()[:5].tolist(),
                                    float(s["gap_item"]), float(s["gap_obj"])))
+    tally.count("schedule", B, exc)
     # the GPU's own offsets must be the exclusive scan of its own lengths
     exp_rs = np.concatenate([[0], np.cumsum(L.astype(np.int64) + 1)[:-1]])
     if not np.array_equal(gpu["row_start"], exp_rs):
@@ -126,15 +132,16 @@ def compare_verify(inp, draft_oracle, gpu_draft, gpu, verify_len, requests, tall
     for idx, b in enumerate(requests):
         Lb = int(verify_len[b])
         margins = vo["accept_margin"][idx]
-        tally.decisions += len(margins)
         tally.flagged += int(sum(m < MARGIN for m in margins))
         ao, ag = int(vo["accepted"][idx]), int(acc_g[idx])
+        exc = 0
         if ao != ag:
             j = min(ao, ag)  # first position where the decisions differ (0-based)
             if j < len(margins) and margins[j] < MARGIN:
-                tally.excused += 1
+                exc = 1
             else:
                 tally.failures.append(("accepted", int(b), ao, ag, margins[j] if j < len(margins) else None))
+        tally.count("accept", len(margins), exc)
         if not (1 <= gpu["n_out"][idx] <= Lb + 1) or gpu["n_out"][idx] != ag + 1:
             tally.failures.append(("n_out", int(b), int(gpu["n_out"][idx]), ag))
         if not np.array_equal(gpu["out_tokens"][idx, :ag], gpu_draft["tokens"][idx, :ag]):
@@ -146,15 +153,16 @@ def compare_verify(inp, draft_oracle, gpu_draft, gpu, verify_len, requests, tall
                         gpu_draft["tokens"], verify_len, inp["u_accept"], inp["u_resample"],
                         forced_accepted=_full(acc_g, requests, B), requests=requests)
     for idx, b in enumerate(requests):
-        tally.decisions += 1
         m = vo2["final_margin"][idx]
         tally.flagged += int(m < MARGIN)
         fg = int(gpu["out_tokens"][idx, acc_g[idx]])
+        exc = 0
         if fg != int(vo2["final"][idx]):
             if m < MARGIN:
-                tally.excused += 1
+                exc = 1
             else:
                 tally.failures.append(("final", int(b), int(vo2["final"][idx]), fg, float(m), vo2["final_mode"][idx]))
+        tally.count("final", 1, exc)
     return vo2
 
 
@@ -164,14 +172,16 @@ def _full(vals, requests, B):
     return out
 
 
-def gpu_round(inp, requests=None, packed=False):
-    """Run draft -> schedule -> verify through the library; numpy outputs."""
+def gpu_round(inp, requests=None, packed=False, bufs=None):
+    """Run draft -> schedule -> verify through the library; numpy outputs.
+    `bufs` (optional) reuses the outputs and workspace of an earlier round."""
     from speculative_decoding_semi_b200 import round as rnd
 
     B, K, V = inp["base"].shape
     r = inp["A"].shape[1]
     d = rnd.to_device(inp)
-    bufs = rnd.RoundBuffers(B, K, V, r)
+    if bufs is None:
+        bufs = rnd.RoundBuffers(B, K, V, r)
     rnd.draft(d, bufs)
     rnd.schedule(d, bufs)
     if packed:
@@ -190,7 +200,7 @@ def gpu_round(inp, requests=None, packed=False):
     take = lambda t: t.index_select(0, ridx).cpu().numpy()
     out = {
         "draft": {"tokens": take(bufs.draft_tokens), "q_tok": take(bufs.q_tok), "lse_q": take(bufs.lse_q),
-                  "z": take(bufs.z) if len(reqs) * K * V <= 64 * 8 * 151936 else None},
+                  "z": take(bufs.z) if len(reqs) * K * V <= 64 * 16 * 151936 else None},
         "schedule": {"verify_len": bufs.verify_len.cpu().numpy(), "survival": bufs.survival.cpu().numpy(),
                      "row_start": bufs.row_start.cpu().numpy(), "n_tokens": bufs.n_tokens.cpu().numpy()[0]},
         "verify": {"accepted": take(bufs.accepted), "out_tokens": take(bufs.out_tokens), "n_out": take(bufs.n_out)},
@@ -198,10 +208,10 @@ def gpu_round(inp, requests=None, packed=False):
     return out
 
 
-def check_round(inp, requests=None, packed=False, tally: Tally | None = None, check_z=True):
+def check_round(inp, requests=None, packed=False, tally: Tally | None = None, check_z=True, bufs=None):
     B = inp["base"].shape[0]
     reqs = np.arange(B) if requests is None else np.asarray(requests)
-    g = gpu_round(inp, reqs, packed=packed)
+    g = gpu_round(inp, reqs, packed=packed, bufs=bufs)
     t = Tally() if tally is None else tally
     d = compare_draft(inp, g["draft"], reqs, t, check_z=check_z and g["draft"]["z"] is not None)
     compare_schedule(inp, g["schedule"], t)
