@@ -324,6 +324,18 @@ __device__ __forceinline__ void fill_exp_table(double* t16, int tid) {
   if (tid < 16) t16[tid] = exp2(static_cast<double>(tid) / 16.0);
 }
 
+// max / min that return NaN when either input is NaN (PTX .NaN form).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ float fmin_nan(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // e^(zh + zl) in fp64, for an fp32 value zh and a small fp32 correction zl
 // (the rounding error of zh, |zl| <= ulp(zh)). Table-driven, after Tang's
 // method: zh = n ln2/16 + r with n the integer nearest zh 16/ln2, so that
@@ -334,20 +346,21 @@ __device__ __forceinline__ void fill_exp_table(double* t16, int tid) {
 // power (truncation < 2e-13) in fp32, whose rounding moves 1 + p by ~3e-9;
 // the last step is one fp64 FMA by the exact 2^(n>>4) 2^((n&15)/16). The
 // result's relative error is ~5e-9 for |zh| < 30 (against ~1e-7 for an fp32
-// exponential of an fp32-rounded argument). zh < -708 gives 0, zh > 709
-// gives +inf, NaN propagates.
+// exponential of an fp32-rounded argument). Branch-free: zh is clamped to
+// [-708, 709] (so a row far outside fp64's range has a sum outside
+// [1e-280, 1e280] and is redrawn by its caller with its own maximum), and a
+// NaN zh gives NaN.
 __device__ __forceinline__ double exp_fine(float zh, float zl, const double* t16) {
   constexpr float kInvC = 23.083120654223414f;     // 16 / ln 2
   constexpr float kC1 = 0.0433349609375f;          // 710 * 2^-14
   constexpr float kC2 = -1.326215250341961e-05f;   // ln2/16 - kC1
-  if (!(zh >= -708.f)) return zh != zh ? static_cast<double>(zh) : 0.0;
-  if (zh > 709.f) return static_cast<double>(INFINITY);
-  // n = zh 16/ln2 rounded to the nearest integer, by adding 1.5 * 2^23 in one
+  const float x = fmin_nan(fmax_nan(zh, -708.f), 709.f);
+  // n = x 16/ln2 rounded to the nearest integer, by adding 1.5 * 2^23 in one
   // rounding (exact product): the integer lands in the low mantissa bits
-  const float tn = fmaf(zh, kInvC, 12582912.f);
+  const float tn = fmaf(x, kInvC, 12582912.f);
   const float n = __fsub_rn(tn, 12582912.f);
   const int ni = __float_as_int(tn) - 0x4B400000;
-  float r = fmaf(-n, kC1, zh);
+  float r = fmaf(-n, kC1, x);
   r = fmaf(-n, kC2, r);
   r = __fadd_rn(r, zl);
   float q = fmaf(r, 1.f / 120.f, 1.f / 24.f);
@@ -357,9 +370,84 @@ __device__ __forceinline__ double exp_fine(float zh, float zl, const double* t16
   const float p = __fmul_rn(q, r);
   const double t = t16[ni & 15];
   // t is in [1, 2); adding (n >> 4) to its exponent field scales it by
-  // 2^(n>>4), within the normal range for |zh| <= 709
+  // 2^(n>>4), within the normal range for |x| <= 709
   const double ts = __hiloint2double(__double2hiint(t) + (ni >> 4) * (1 << 20), __double2loint(t));
   return fma(ts, static_cast<double>(p), ts);
+}
+
+// ------------------------------------------- packed fp32 pairs (sm_100)
+// Two fp32 values in one 64-bit register, for the .f32x2 forms of add, sub,
+// mul and fma (one instruction, two results, each rounded as its scalar form).
+struct F2 {
+  unsigned long long v;
+};
+__device__ __forceinline__ F2 f2(float a, float b) {
+  F2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float f2_lo(F2 x) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x.v));
+  return a;
+}
+__device__ __forceinline__ float f2_hi(F2 x) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(x.v));
+  return b;
+}
+__device__ __forceinline__ F2 add2(F2 a, F2 b) {
+  F2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ F2 sub2(F2 a, F2 b) {
+  F2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
+  F2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
+  F2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return r;
+}
+
+// TwoSum of two pairs: s = fl(a + b) and the exact rounding error e, a + b = s + e.
+__device__ __forceinline__ void two_sum2(F2 a, F2 b, F2* s, F2* e) {
+  *s = add2(a, b);
+  const F2 bv = sub2(*s, a);
+  *e = add2(sub2(a, sub2(*s, bv)), sub2(b, bv));
+}
+
+// exp_fine of two values at once: the fp32 steps in pairs, the table lookup,
+// exponent scaling and final fp64 FMA per value (same arithmetic, same result).
+__device__ __forceinline__ void exp_fine2(F2 zh, F2 zl, const double* t16, double* w0, double* w1) {
+  const F2 kInvC = f2(23.083120654223414f, 23.083120654223414f);
+  const F2 kMagic = f2(12582912.f, 12582912.f);
+  const F2 kNC1 = f2(-0.0433349609375f, -0.0433349609375f);
+  const F2 kNC2 = f2(1.326215250341961e-05f, 1.326215250341961e-05f);
+  const F2 x = f2(fmin_nan(fmax_nan(f2_lo(zh), -708.f), 709.f), fmin_nan(fmax_nan(f2_hi(zh), -708.f), 709.f));
+  const F2 tn = fma2(x, kInvC, kMagic);
+  const F2 n = sub2(tn, kMagic);
+  F2 r = fma2(n, kNC1, x);
+  r = fma2(n, kNC2, r);
+  r = add2(r, zl);
+  F2 q = fma2(r, f2(1.f / 120.f, 1.f / 120.f), f2(1.f / 24.f, 1.f / 24.f));
+  q = fma2(q, r, f2(1.f / 6.f, 1.f / 6.f));
+  q = fma2(q, r, f2(0.5f, 0.5f));
+  q = fma2(q, r, f2(1.f, 1.f));
+  const F2 p = mul2(q, r);
+  const int n0 = __float_as_int(f2_lo(tn)) - 0x4B400000, n1 = __float_as_int(f2_hi(tn)) - 0x4B400000;
+  const double t0 = t16[n0 & 15], t1 = t16[n1 & 15];
+  const double s0 = __hiloint2double(__double2hiint(t0) + (n0 >> 4) * (1 << 20), __double2loint(t0));
+  const double s1 = __hiloint2double(__double2hiint(t1) + (n1 >> 4) * (1 << 20), __double2loint(t1));
+  *w0 = fma(s0, static_cast<double>(f2_lo(p)), s0);
+  *w1 = fma(s1, static_cast<double>(f2_hi(p)), s1);
 }
 
 // fp32 -> bf16 bits, round to nearest even (finite inputs).

@@ -645,6 +645,13 @@ __global__ void __maxnreg__(96)
     }
     float* ring = reinterpret_cast<float*>(smem + Ly.ring + warp * p.nbs * kBoxBytes);
     uint16_t* lobox = reinterpret_cast<uint16_t*>(smem + Ly.lo + warp * kLoBoxBytes);
+    // element offsets of (row c, vocabulary lane) in the two swizzled boxes,
+    // for each value of c & 7 and (c / 2) & 3
+    int zsw[8], losw[4];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) zsw[x] = (((lane >> 2) ^ x) << 2) + (lane & 3);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) losw[x] = (((lane >> 3) ^ x) << 3) + (lane & 7);
     uint64_t* rfull = bars.base_full(warp * kMaxRingSlots);
     Items L;
     L.p = &p;
@@ -725,19 +732,26 @@ __global__ void __maxnreg__(96)
                                          static_cast<uint32_t>(slot * p.slot_stride + col0),
                                      rg);
                   tmem_ld_wait();
-                  // z = base + bias in place (lane = vocabulary row, c = request),
+                  // z = base + bias in place (lane = vocabulary row v, c = request),
                   // its rounding error by TwoSum into the bf16 box (its upper
-                  // 16 bits: ~2^-8 of an error that is itself below ulp(z));
-                  // the previous sub-chunk's reads of that box are done first
+                  // 16 bits: ~2^-8 of an error that is itself below ulp(z)).
+                  // The box is [c][32 v] fp32 with TMA's 128-byte swizzle
+                  // (16-byte chunk v/4 of row c at chunk (v/4) ^ (c & 7)); the
+                  // error box is [c][32 v] u16 with chunk v/8 of row c at
+                  // (v/8) ^ ((c/2) & 3). The previous sub-chunk's reads of the
+                  // error box are done first.
                   __syncwarp();
 #pragma unroll
-                  for (int c = 0; c < kSub; ++c) {
-                    const float x0 = box[c * kUnit + lane], y0 = __uint_as_float(rg[c]);
-                    const float sum = __fadd_rn(x0, y0);
-                    const float yv = __fsub_rn(sum, x0);
-                    const float err = __fadd_rn(__fsub_rn(x0, __fsub_rn(sum, yv)), __fsub_rn(y0, yv));
-                    box[c * kUnit + lane] = sum;
-                    lobox[c * kUnit + lane] = static_cast<uint16_t>(__float_as_uint(err) >> 16);
+                  for (int c = 0; c < kSub; c += 2) {
+                    float* zp0 = box + c * kUnit + zsw[c & 7];
+                    float* zp1 = box + (c + 1) * kUnit + zsw[(c + 1) & 7];
+                    F2 sum, err;
+                    two_sum2(f2(*zp0, *zp1), f2(__uint_as_float(rg[c]), __uint_as_float(rg[c + 1])), &sum, &err);
+                    *zp0 = f2_lo(sum);
+                    *zp1 = f2_hi(sum);
+                    lobox[c * kUnit + losw[(c >> 1) & 3]] = static_cast<uint16_t>(__float_as_uint(f2_lo(err)) >> 16);
+                    lobox[(c + 1) * kUnit + losw[((c + 1) >> 1) & 3]] =
+                        static_cast<uint16_t>(__float_as_uint(f2_hi(err)) >> 16);
                   }
                   fence_proxy_async_shared();
                   __syncwarp();
@@ -746,19 +760,32 @@ __global__ void __maxnreg__(96)
                     tma_store_3d(&tm_z, box, v0, i, gbase + col0, pol_first);
                     bulk_commit();
                   }
-                  // the box's sum over its 32 rows for request col0 + (lane & 15):
-                  // lane l reads rows 16 (l >> 4) .. + 15, starting at a row
-                  // rotated by the request so that the 32 lanes hit 32 banks;
-                  // the two halves meet in one shuffle
-                  const int cr = lane & (kSub - 1);
-                  const float* colp = box + cr * kUnit + (lane >> 4) * 16;
-                  const uint16_t* lop = lobox + cr * kUnit + (lane >> 4) * 16;
+                  // the box's sum over its 32 rows for request cr = lane & 15:
+                  // lane l reads rows 16 (l >> 4) .. + 15 of row cr of both
+                  // boxes with 128-bit loads (the swizzles spread each load over
+                  // all banks), and the two halves meet in one shuffle
+                  const int cr = lane & (kSub - 1), hf = lane >> 4;
+                  const float4* zrow4 = reinterpret_cast<const float4*>(box + cr * kUnit);
+                  const uint4* lrow4 = reinterpret_cast<const uint4*>(lobox + cr * kUnit);
                   double us0 = 0.0, us1 = 0.0;
-#pragma unroll 4
-                  for (int k = 0; k < 16; k += 2) {
-                    const int k0 = (k + cr) & 15, k1 = (k + 1 + cr) & 15;
-                    us0 += exp_fine(colp[k0], bf16_bits_to_float(lop[k0]), t16);
-                    us1 += exp_fine(colp[k1], bf16_bits_to_float(lop[k1]), t16);
+#pragma unroll
+                  for (int qq = 0; qq < 2; ++qq) {
+                    const uint4 lv = lrow4[(2 * hf + qq) ^ ((cr >> 1) & 3)];
+                    const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                      const float4 zv = zrow4[(4 * hf + 2 * qq + h2) ^ (cr & 7)];
+                      const uint32_t a = lw[2 * h2], b = lw[2 * h2 + 1];
+                      double w0, w1, w2, w3;
+                      exp_fine2(f2(zv.x, zv.y), f2(__uint_as_float(a << 16), __uint_as_float(a & 0xffff0000u)), t16,
+                                &w0, &w1);
+                      exp_fine2(f2(zv.z, zv.w), f2(__uint_as_float(b << 16), __uint_as_float(b & 0xffff0000u)), t16,
+                                &w2, &w3);
+                      us0 += w0;
+                      us1 += w1;
+                      us0 += w2;
+                      us1 += w3;
+                    }
                   }
                   double us = us0 + us1;
                   us += __shfl_xor_sync(0xffffffffu, us, 16);
@@ -908,7 +935,7 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
     cuuint32_t box[3] = {static_cast<cuuint32_t>(kUnit), 1, static_cast<cuuint32_t>(kSub)};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
   if (!enc3(&tm_base, a.base) || !enc3(&tm_z, a.z)) return cudaErrorInvalidValue;

@@ -67,11 +67,14 @@ def workload(key) -> Workload:
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (round to nearest, ties to even); returns uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    rounded = (u + 0x7FFF + lsb) >> 16
-    return rounded.astype(np.uint16)
+    """Round fp32 to bf16 (round to nearest, ties to even); returns uint16 bits.
+    Finite inputs only (the uint32 sum cannot carry out of 32 bits for them)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -133,13 +136,28 @@ def custom(like, **sizes) -> Workload:
     return dataclasses.replace(workload(like), **sizes)
 
 
-def make_round(key, seed: int | None = None, with_target: bool = True) -> dict:
+def make_factors(key, seed: int | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """The Markov factors (A [V,r], Bf [r,V]) that make_round draws for this seed."""
+    w = workload(key)
+    ss = np.random.SeedSequence(w.seed if seed is None else seed)
+    rngs = dict(zip(STREAMS, (np.random.default_rng(s) for s in ss.spawn(len(STREAMS)))))
+    A = _normal(rngs["A"], (w.V, w.r), w.factor_std)
+    Bf = _normal(rngs["Bf"], (w.r, w.V), w.factor_std)
+    if w.factor_dtype == "bf16":
+        A, Bf = f32_to_bf16_bits(A), f32_to_bf16_bits(Bf)
+    return A, Bf
+
+
+def make_round(key, seed: int | None = None, with_target: bool = True, factors=None) -> dict:
     """All inputs of one round of the given workload, as host numpy arrays.
 
     Keys: base [B,K,V] f32; A [V,r], Bf [r,V] (f32, or uint16 bf16 bits);
     anchor [B] i32; u_draft [B,K], u_accept [B,K], u_resample [B] f32;
     conf [B,K] f32; temps [K] f32; profile [n_prof] f32; sigma [B] f32;
     target [B,K+1,V] f32 (dense: row rho of request b at b*(K+1)+rho).
+    `factors` (A, Bf) replaces the seed's own factors: the Markov head's
+    weights, which stay fixed while the per-round inputs change; every other
+    stream is the seed's.
     """
     w = workload(key)
     ss = np.random.SeedSequence(w.seed if seed is None else seed)
@@ -147,10 +165,14 @@ def make_round(key, seed: int | None = None, with_target: bool = True) -> dict:
     B, K, V, r = w.B, w.K, w.V, w.r
     out = {"workload": w}
     out["base"] = _normal(rngs["base"], (B, K, V), 2.0)
-    A = _normal(rngs["A"], (V, r), w.factor_std)
-    Bf = _normal(rngs["Bf"], (r, V), w.factor_std)
-    if w.factor_dtype == "bf16":
-        A, Bf = f32_to_bf16_bits(A), f32_to_bf16_bits(Bf)
+    if factors is None:
+        A = _normal(rngs["A"], (V, r), w.factor_std)
+        Bf = _normal(rngs["Bf"], (r, V), w.factor_std)
+        if w.factor_dtype == "bf16":
+            A, Bf = f32_to_bf16_bits(A), f32_to_bf16_bits(Bf)
+    else:
+        A, Bf = factors
+        assert A.shape == (V, r) and Bf.shape == (r, V)
     out["A"], out["Bf"] = A, Bf
     sigma = _sigma(w, rngs["sigma"])
     out["sigma"] = sigma

@@ -141,10 +141,14 @@ def test_full_size_mixed_packed():
 def test_full_size_seed_volume(key, seeds, sample):
     """More seeds of every full-size workload (with the ones above: 20 of
     qwen3, 201 of latency, 3 of highconc and of mixed), the excused near-ties
-    pooled over them; z is compared on the first seeds."""
+    pooled over them; z is compared on the first seeds. The Markov factors are
+    model weights: drawn once per workload (from its own seed), while every
+    per-round input (logits, uniforms, anchors, confidences) comes from each
+    round's seed."""
     t = parity.Tally()
+    factors = synth.make_factors(key)
     for k in range(seeds):
-        inp = synth.make_round(key, seed=7000 + k)
+        inp = synth.make_round(key, seed=7000 + k, factors=factors)
         B = inp["base"].shape[0]
         parity.check_round(inp, requests=_sample(B, sample, k + 1), tally=t, check_z=k < 2)
     t.check(f"{key} x{seeds}")
