@@ -30,7 +30,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["bf16_to_f64", "softmax", "icdf", "markov_bias", "draft_step", "draft",
-           "survival", "schedule", "verify", "run_round"]
+           "survival", "schedule", "verify", "run_round", "calibrate"]
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -283,3 +283,45 @@ def run_round(inp: dict, requests=None) -> dict:
     v = verify(rows, rs, d["z"], d["lse"], d["q_tok"], d["t"], s["verify_len"],
                inp["u_accept"], inp["u_resample"], requests=reqs)
     return {"draft": d, "survival": P, "schedule": s, "verify": v, "requests": reqs}
+
+
+def calibrate(conf, temps, verify_len, accepted, eta: float, t_min: float, t_max: float) -> np.ndarray:
+    """One online step of sequential temperature scaling from a round's outcome.
+
+    [QbitAI] section "online drafter calibration": the confidence head is
+    over-confident, so its scores are post-processed by sequential temperature
+    scaling, and the calibration runs online, correcting itself from the
+    acceptance actually observed on the current workload; [Thread] item 10
+    (observe the drafter at run time and adjust the thresholds dynamically);
+    [Essay] section "the hard step ...": the confidence is the chance that a
+    position survives given that every earlier draft passed.
+    Reading: position j's temperature T_j is the scale of a logistic model
+    s = sigmoid(c / T_j) of that conditional survival, and temperature scaling
+    fits it by the negative log-likelihood of observed outcomes. The
+    observations of position j in a round are the requests that reached it
+    (drafts 1..j-1 accepted) and verified it (j <= L_b), with outcome
+    y = 1 if draft j was accepted. Online, each round takes one gradient step
+    on theta_j = 1 / T_j with the mean gradient over those observations:
+        g_j = (1/n_j) sum_b (sigmoid(c_bj theta_j) - y_bj) c_bj
+        theta_j <- theta_j - eta g_j,  T_j = clamp(1 / theta_j, t_min, t_max).
+    A position with no observation keeps its temperature. Returns the new
+    temperatures (fp64).
+    """
+    c = np.asarray(conf, np.float64)
+    T = np.asarray(temps, np.float64).copy()
+    L = np.asarray(verify_len, np.int64)
+    acc = np.asarray(accepted, np.int64)
+    B, K = c.shape
+    for j in range(1, K + 1):
+        reached = (acc >= j - 1) & (L >= j)
+        n = int(reached.sum())
+        if n == 0:
+            continue
+        theta = 1.0 / T[j - 1]
+        cj = c[reached, j - 1]
+        y = (acc[reached] >= j).astype(np.float64)
+        s = 1.0 / (1.0 + np.exp(-cj * theta))
+        g = float(np.sum((s - y) * cj)) / n
+        theta = theta - eta * g
+        T[j - 1] = np.clip(1.0 / theta, t_min, t_max) if theta > 0 else t_max
+    return T
