@@ -135,6 +135,47 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
                             dspark_stream_t stream);
 
 /*
+ * Online calibration of the sequential temperatures from one round's outcome.
+ * [QbitAI] section "online drafter calibration" (the confidence scores are
+ * post-processed by sequential temperature scaling, and the calibration runs
+ * online from the acceptance observed on the workload); [Thread] item 10;
+ * [Essay] section "the hard step ..." (survival given that earlier drafts passed).
+ *
+ * Position j's temperature is the scale of the logistic survival model
+ * sigmoid(c / T_j). The observations of position j are the requests with
+ * accepted[b] >= j-1 (they reached it) and verify_len[b] >= j (they verified
+ * it), with outcome y = (accepted[b] >= j). One step on theta_j = 1 / T_j:
+ *   g_j = (1/n_j) sum_b (sigmoid(conf[b,j] theta_j) - y_bj) conf[b,j]
+ *   theta_j -= eta g_j;  temps[j] = clamp(1 / theta_j, t_min, t_max)
+ * (a non-positive theta_j gives t_max); positions nobody reached keep their
+ * temperature. Sums in fp64 in a fixed order.
+ *
+ * conf_logits [B,K] f32; verify_len, accepted [B] i32 (as dspark_schedule and
+ * dspark_verify produced them); temps [K] f32, updated in place, so the next
+ * dspark_schedule on the stream uses the calibrated values. eta >= 0,
+ * 0 < t_min <= t_max. The workspace is used for its error word only (a
+ * verify_len outside [0,K] or an accepted count outside [0,L_b] is recorded
+ * and that request skipped).
+ */
+dspark_status dspark_calibrate(const float* conf_logits, const int32_t* verify_len, const int32_t* accepted,
+                               int B, int K, float eta, float t_min, float t_max, float* temps,
+                               void* workspace, size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * The next round's anchors from this round's output: anchor[b] becomes the
+ * last token request b emitted, out_tokens[b, n_out[b]-1] (the token the next
+ * draft block follows). With dspark_calibrate this lets rounds follow one
+ * another on the device with no host round trip ([QbitAI] section
+ * "variable-length drafts and hardware-aware scheduling": the whole logic on
+ * the GPU). out_tokens [B,K+1], n_out [B] i32 as dspark_verify wrote them;
+ * anchor [B] i32 is overwritten. An n_out outside [1,K+1] is recorded in the
+ * workspace's error word and leaves that anchor unchanged.
+ */
+dspark_status dspark_advance_anchor(const int32_t* out_tokens, const int32_t* n_out, int B, int K,
+                                    int32_t* anchor, void* workspace, size_t ws_bytes,
+                                    dspark_stream_t stream);
+
+/*
  * dspark_schedule without a workspace, for callers that cannot allocate
  * device memory (their allocator belongs to another framework, they run inside
  * stream capture, or their hot path forbids cudaMalloc). The pages describe no

@@ -51,6 +51,11 @@ def _load() -> ctypes.CDLL:
     lib.dspark_read_device_error.restype = I
     lib.dspark_schedule_static.argtypes = [P, P, P, I, I, I, P, P, P, P, S]
     lib.dspark_schedule_static.restype = I
+    F = ctypes.c_float
+    lib.dspark_calibrate.argtypes = [P, P, P, I, I, F, F, F, P, P, Z, S]
+    lib.dspark_calibrate.restype = I
+    lib.dspark_advance_anchor.argtypes = [P, P, I, I, P, P, Z, S]
+    lib.dspark_advance_anchor.restype = I
     lib.dspark_set_wait_budget.argtypes = [P, ctypes.c_uint32, S]
     lib.dspark_set_wait_budget.restype = I
     lib.dspark_inject_stall.argtypes = [P, I, ctypes.c_uint32, S]
@@ -165,6 +170,28 @@ def dspark_verify(target_logits, row_start, z, lse_q, q_tok, draft_tokens, verif
         _ptr(n_out, "n_out", torch.int32, B), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
         _stream(stream))
     _check("dspark_verify", st)
+
+
+def dspark_calibrate(conf_logits, verify_len, accepted, temps, workspace, eta: float, t_min: float, t_max: float,
+                     stream=None) -> None:
+    """One online step of the sequential temperatures (temps updated in place)."""
+    B, K = conf_logits.shape
+    st = lib.dspark_calibrate(
+        _ptr(conf_logits, "conf_logits", torch.float32), _ptr(verify_len, "verify_len", torch.int32, B),
+        _ptr(accepted, "accepted", torch.int32, B), B, K, float(eta), float(t_min), float(t_max),
+        _ptr(temps, "temps", torch.float32, K), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+        _stream(stream))
+    _check("dspark_calibrate", st)
+
+
+def dspark_advance_anchor(out_tokens, n_out, anchor, workspace, stream=None) -> None:
+    """anchor[b] = out_tokens[b, n_out[b]-1], for the next round."""
+    B, K1 = out_tokens.shape
+    st = lib.dspark_advance_anchor(
+        _ptr(out_tokens, "out_tokens", torch.int32), _ptr(n_out, "n_out", torch.int32, B), B, K1 - 1,
+        _ptr(anchor, "anchor", torch.int32, B), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+        _stream(stream))
+    _check("dspark_advance_anchor", st)
 
 
 DSPARK_INJECT_NONE, DSPARK_INJECT_DRAFT_SLICE_SUMS, DSPARK_INJECT_VERIFY_BARRIER = 0, 1, 2

@@ -1,17 +1,19 @@
-"""One DSpark round on the GPU through the C ABI: draft -> schedule -> verify.
+"""DSpark rounds on the GPU through the C ABI: draft -> schedule -> verify.
 
 `RoundBuffers` owns the device outputs and the workspace of one round shape;
 `run_round` enqueues the three library calls on one stream without any host
 synchronisation (the scheduler's verify lengths and row offsets stay on the
-device and feed the verification directly).
+device and feed the verification directly). `run_rounds` chains rounds on the
+device (online temperature calibration and the next anchors included), as a
+plain stream of launches or one captured CUDA graph.
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-from .binding import (dspark_markov_draft, dspark_schedule, dspark_verify, dspark_workspace_bytes,
-                      dspark_workspace_init)
+from .binding import (dspark_advance_anchor, dspark_calibrate, dspark_markov_draft, dspark_schedule, dspark_verify,
+                      dspark_workspace_bytes, dspark_workspace_init)
 
 
 def to_device(inputs: dict, device="cuda") -> dict:
@@ -75,3 +77,73 @@ def run_round(d: dict, bufs: RoundBuffers, stream=None):
     draft(d, bufs, stream)
     schedule(d, bufs, stream)
     verify(d, bufs, stream=stream)
+
+
+class RoundState:
+    """What carries from one round to the next on the device: the anchors
+    (the last token each request emitted) and the calibrated temperatures."""
+
+    def __init__(self, anchor: torch.Tensor, temps: torch.Tensor):
+        self.anchor = anchor.clone()
+        self.temps = temps.clone()
+
+
+HISTORY = {"anchor": ("B",), "temps": ("K",), "draft_tokens": ("B", "K"), "q_tok": ("B", "K"),
+           "lse_q": ("B", "K"), "verify_len": ("B",), "survival": ("B", "K"), "row_start": ("B",),
+           "n_tokens": (1,), "accepted": ("B",), "out_tokens": ("B", "K+1"), "n_out": ("B",)}
+
+
+def run_rounds(inputs: list, bufs: RoundBuffers, state: RoundState, rounds: int, calibrate=None,
+               record: bool = True, graph: bool = False, stream=None) -> dict:
+    """`rounds` rounds back to back on one stream, with no host synchronisation:
+    draft -> schedule -> verify -> (calibrate) -> next anchors. Round r reads
+    inputs[r % len(inputs)] (device dicts from to_device; in a serving system
+    the backbone and target forward passes would refill these between rounds)
+    and the anchors and temperatures in `state`, which the round updates.
+    calibrate = (eta, t_min, t_max) turns on the online temperature step.
+    With record=True each round's state and outputs are copied into history
+    tensors [rounds, ...] (device-to-device). With graph=True the rounds are
+    captured once as a CUDA graph and replayed; the graph is returned in the
+    result under "graph" so that it can be replayed again.
+    """
+    B, K = bufs.B, bufs.K
+    dims = {"B": B, "K": K, "K+1": K + 1}
+    hist = {}
+    if record:
+        for name, shape in HISTORY.items():
+            ref = state.anchor if name == "anchor" else state.temps if name == "temps" else getattr(bufs, name)
+            hist[name] = torch.empty((rounds,) + tuple(dims.get(s, s) for s in shape), dtype=ref.dtype,
+                                     device=ref.device)
+
+    def body(s):
+        for r in range(rounds):
+            d = inputs[r % len(inputs)]
+            if record:
+                hist["anchor"][r].copy_(state.anchor, non_blocking=True)
+                hist["temps"][r].copy_(state.temps, non_blocking=True)
+            dspark_markov_draft(d["base"], d["A"], d["Bf"], state.anchor, d["u_draft"], bufs.draft_tokens,
+                                bufs.q_tok, bufs.lse_q, bufs.z, bufs.workspace, s)
+            dspark_schedule(d["conf"], state.temps, d["profile"], bufs.verify_len, bufs.survival, bufs.row_start,
+                            bufs.n_tokens, bufs.workspace, s)
+            dspark_verify(d["target"], d["row_start_dense"], bufs.z, bufs.lse_q, bufs.q_tok, bufs.draft_tokens,
+                          bufs.verify_len, d["u_accept"], d["u_resample"], bufs.accepted, bufs.out_tokens, bufs.n_out,
+                          bufs.workspace, s)
+            if record:
+                for name in HISTORY:
+                    if name not in ("anchor", "temps"):
+                        hist[name][r].copy_(getattr(bufs, name), non_blocking=True)
+            if calibrate is not None:
+                eta, t_min, t_max = calibrate
+                dspark_calibrate(d["conf"], bufs.verify_len, bufs.accepted, state.temps, bufs.workspace, eta, t_min,
+                                 t_max, s)
+            dspark_advance_anchor(bufs.out_tokens, bufs.n_out, state.anchor, bufs.workspace, s)
+
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            body(torch.cuda.current_stream())
+        g.replay()
+        hist["graph"] = g
+    else:
+        body(stream)
+    return hist

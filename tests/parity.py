@@ -208,12 +208,18 @@ def gpu_round(inp, requests=None, packed=False, bufs=None):
     return out
 
 
+def compare_round(inp, g, reqs, tally: Tally, check_z=True):
+    """Compare one round's GPU outputs `g` (as gpu_round returns them) with
+    the oracle on the same inputs."""
+    d = compare_draft(inp, g["draft"], reqs, tally, check_z=check_z and g["draft"].get("z") is not None)
+    compare_schedule(inp, g["schedule"], tally)
+    compare_verify(inp, d, g["draft"], g["verify"], g["schedule"]["verify_len"], reqs, tally)
+
+
 def check_round(inp, requests=None, packed=False, tally: Tally | None = None, check_z=True, bufs=None):
     B = inp["base"].shape[0]
     reqs = np.arange(B) if requests is None else np.asarray(requests)
     g = gpu_round(inp, reqs, packed=packed, bufs=bufs)
     t = Tally() if tally is None else tally
-    d = compare_draft(inp, g["draft"], reqs, t, check_z=check_z and g["draft"]["z"] is not None)
-    compare_schedule(inp, g["schedule"], t)
-    compare_verify(inp, d, g["draft"], g["verify"], g["schedule"]["verify_len"], reqs, t)
+    compare_round(inp, g, reqs, t, check_z=check_z)
     return t, g
