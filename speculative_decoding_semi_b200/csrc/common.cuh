@@ -450,6 +450,57 @@ __device__ __forceinline__ void exp_fine2(F2 zh, F2 zl, const double* t16, doubl
   *w1 = fma(s1, static_cast<double>(f2_hi(p)), s1);
 }
 
+// e^(x + y) for two pairs, where zh = fl(x + y) is already formed: the same
+// table-driven steps as exp_fine, with the reduced argument built from x and y
+// themselves, r = (x - n ln2/16) + y, so that the rounding error of zh never
+// enters (x is the base logit, y the small Markov bias). n comes from the
+// clamped zh; when zh is clamped the argument is shifted with it.
+__device__ __forceinline__ void exp_sum2(F2 x, F2 y, F2 zh, const double* t16, double* w0, double* w1) {
+  const F2 kInvC = f2(23.083120654223414f, 23.083120654223414f);
+  const F2 kMagic = f2(12582912.f, 12582912.f);
+  const F2 kNC1 = f2(-0.0433349609375f, -0.0433349609375f);
+  const F2 kNC2 = f2(1.326215250341961e-05f, 1.326215250341961e-05f);
+  const F2 zc = f2(fmin_nan(fmax_nan(f2_lo(zh), -708.f), 709.f), fmin_nan(fmax_nan(f2_hi(zh), -708.f), 709.f));
+  const F2 xs = add2(x, sub2(zc, zh));   // x itself unless zh was clamped
+  const F2 tn = fma2(zc, kInvC, kMagic);
+  const F2 n = sub2(tn, kMagic);
+  F2 r = fma2(n, kNC1, xs);
+  r = fma2(n, kNC2, r);
+  r = add2(r, y);
+  F2 q = fma2(r, f2(1.f / 120.f, 1.f / 120.f), f2(1.f / 24.f, 1.f / 24.f));
+  q = fma2(q, r, f2(1.f / 6.f, 1.f / 6.f));
+  q = fma2(q, r, f2(0.5f, 0.5f));
+  q = fma2(q, r, f2(1.f, 1.f));
+  const F2 p = mul2(q, r);
+  const int n0 = __float_as_int(f2_lo(tn)) - 0x4B400000, n1 = __float_as_int(f2_hi(tn)) - 0x4B400000;
+  const double t0 = t16[n0 & 15], t1 = t16[n1 & 15];
+  const double s0 = __hiloint2double(__double2hiint(t0) + (n0 >> 4) * (1 << 20), __double2loint(t0));
+  const double s1 = __hiloint2double(__double2hiint(t1) + (n1 >> 4) * (1 << 20), __double2loint(t1));
+  *w0 = fma(s0, static_cast<double>(f2_lo(p)), s0);
+  *w1 = fma(s1, static_cast<double>(f2_hi(p)), s1);
+}
+
+// Sum over the 32 lanes of a warp of 16 values per lane, v[c] for c = 0..15:
+// a halving exchange (lanes split the values at each step and add what their
+// partner sends), then one final exchange. Lane l returns the total of
+// v[l >> 1] (lanes 2c and 2c + 1 both hold the total of value c). 15 paired
+// exchanges and one more: about 7 instructions per value.
+__device__ __forceinline__ double warp_transpose_sum16(double (&v)[16], int lane) {
+#pragma unroll
+  for (int step = 0; step < 4; ++step) {
+    const int half = 8 >> step;           // values kept after this step
+    const int bit = 16 >> step;           // partner lane distance
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const double send = upper ? v[i] : v[i + half];
+      const double keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
 // fp32 -> bf16 bits, round to nearest even (finite inputs).
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
   const unsigned u = __float_as_uint(x);

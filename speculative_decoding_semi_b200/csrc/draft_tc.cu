@@ -31,11 +31,13 @@
 //              group's tokens before releasing the next position.
 // The epilogue streams base and z through per-warp TMA rings (L2 evict-first)
 // that run ahead across positions, since they do not depend on the tokens.
-// Weights. z = base + bias is rounded to fp32 for the output; its rounding
-// error (TwoSum, kept in bf16, ~1e-9 of z) is carried into the weight, which
-// is exp(z) in fp64 (exp_fine, relative error ~5e-9) with a fixed shift of 0,
-// so the sums that place the draw differ from exact ones by ~1e-10 of the row's
-// mass instead of the ~3e-9 an fp32 exponential of the rounded z would give.
+// Weights. z = base + bias is rounded to fp32 for the output, but the weight
+// is exp(base + bias) in fp64 (exp_sum2: the reduced argument is built from
+// base and bias, so z's rounding never enters; relative error ~5e-9) with a
+// fixed shift of 0, and the 32 rows of a unit are summed across the warp's
+// lanes in fp64 (warp_transpose_sum16). The sums that place the draw then
+// differ from exact ones by ~1e-10 of the row's mass instead of the ~3e-9 an
+// fp32 exponential of the rounded z would give.
 // The last level of the search reads the stored fp32 z; the error there is
 // confined to one 32-row unit. A row whose sum leaves [1e-280, 1e280] is
 // redone by the selector with its exact maximum as the shift. Every wait is
@@ -75,7 +77,6 @@ constexpr int kMaxRingSlots = 8;
 constexpr int kMaxAccSlots = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarBytes = 2048;
-constexpr int kLoBoxBytes = kSub * kUnit * 2;    // bf16 rounding errors of one z box
 constexpr int kSubPerWarp = kMaxGroup / kSub / 4;  // sub-chunks of a group per epilogue warp
 constexpr double kSumLo = 1e-280, kSumHi = 1e280;  // row sums handled with the fixed shift
 
@@ -97,7 +98,7 @@ struct TcParams {
 };
 
 struct Layout {
-  int bf, brows, ring, lo, part, bar, tab, misc, total;
+  int bf, brows, ring, part, bar, tab, misc, total;
 };
 
 __host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs, int part_bytes) {
@@ -105,8 +106,7 @@ __host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs,
   L.bf = 0;
   L.brows = L.bf + nbf * kBfStageBytes;
   L.ring = L.brows + ((brows_bytes + 1023) / 1024) * 1024;
-  L.lo = L.ring + kEpiWarps * nbs * kBoxBytes;
-  L.part = L.lo + kEpiWarps * kLoBoxBytes;
+  L.part = L.ring + kEpiWarps * nbs * kBoxBytes;
   L.bar = L.part + ((part_bytes + 15) / 16) * 16;
   L.tab = L.bar + kBarBytes;
   L.misc = L.tab + 16 * 8;
@@ -644,14 +644,6 @@ __global__ void __maxnreg__(96)
       prefetch_tmap(&tm_z);
     }
     float* ring = reinterpret_cast<float*>(smem + Ly.ring + warp * p.nbs * kBoxBytes);
-    uint16_t* lobox = reinterpret_cast<uint16_t*>(smem + Ly.lo + warp * kLoBoxBytes);
-    // element offsets of (row c, vocabulary lane) in the two swizzled boxes,
-    // for each value of c & 7 and (c / 2) & 3
-    int zsw[8], losw[4];
-#pragma unroll
-    for (int x = 0; x < 8; ++x) zsw[x] = (((lane >> 2) ^ x) << 2) + (lane & 3);
-#pragma unroll
-    for (int x = 0; x < 4; ++x) losw[x] = (((lane >> 3) ^ x) << 3) + (lane & 7);
     uint64_t* rfull = bars.base_full(warp * kMaxRingSlots);
     Items L;
     L.p = &p;
@@ -705,7 +697,7 @@ __global__ void __maxnreg__(96)
         const int nreal = group_real(p, gr);
         const int hh = half_of(h, gr);
         const int nk = chunks_for(nreal, hh);
-        // lane l < 16 sums column (request) col0 + l of each sub-chunk over the slice
+        // lane 2c sums column (request) col0 + c of each sub-chunk over the slice
         double acc[kSubPerWarp];
 #pragma unroll
         for (int k = 0; k < kSubPerWarp; ++k) acc[k] = 0.0;
@@ -732,26 +724,19 @@ __global__ void __maxnreg__(96)
                                          static_cast<uint32_t>(slot * p.slot_stride + col0),
                                      rg);
                   tmem_ld_wait();
-                  // z = base + bias in place (lane = vocabulary row v, c = request),
-                  // its rounding error by TwoSum into the bf16 box (its upper
-                  // 16 bits: ~2^-8 of an error that is itself below ulp(z)).
-                  // The box is [c][32 v] fp32 with TMA's 128-byte swizzle
-                  // (16-byte chunk v/4 of row c at chunk (v/4) ^ (c & 7)); the
-                  // error box is [c][32 v] u16 with chunk v/8 of row c at
-                  // (v/8) ^ ((c/2) & 3). The previous sub-chunk's reads of the
-                  // error box are done first.
-                  __syncwarp();
+                  // z = base + bias in place (lane = vocabulary row, c = request)
+                  // and its weight exp(base + bias) in fp64, with the reduced
+                  // argument built from base and bias themselves (exp_sum2),
+                  // so that z's fp32 rounding never enters the weight
+                  double wv[kSub];
 #pragma unroll
                   for (int c = 0; c < kSub; c += 2) {
-                    float* zp0 = box + c * kUnit + zsw[c & 7];
-                    float* zp1 = box + (c + 1) * kUnit + zsw[(c + 1) & 7];
-                    F2 sum, err;
-                    two_sum2(f2(*zp0, *zp1), f2(__uint_as_float(rg[c]), __uint_as_float(rg[c + 1])), &sum, &err);
-                    *zp0 = f2_lo(sum);
-                    *zp1 = f2_hi(sum);
-                    lobox[c * kUnit + losw[(c >> 1) & 3]] = static_cast<uint16_t>(__float_as_uint(f2_lo(err)) >> 16);
-                    lobox[(c + 1) * kUnit + losw[((c + 1) >> 1) & 3]] =
-                        static_cast<uint16_t>(__float_as_uint(f2_hi(err)) >> 16);
+                    const F2 x = f2(box[c * kUnit + lane], box[(c + 1) * kUnit + lane]);
+                    const F2 y = f2(__uint_as_float(rg[c]), __uint_as_float(rg[c + 1]));
+                    const F2 zh = add2(x, y);
+                    box[c * kUnit + lane] = f2_lo(zh);
+                    box[(c + 1) * kUnit + lane] = f2_hi(zh);
+                    exp_sum2(x, y, zh, t16, &wv[c], &wv[c + 1]);
                   }
                   fence_proxy_async_shared();
                   __syncwarp();
@@ -760,37 +745,11 @@ __global__ void __maxnreg__(96)
                     tma_store_3d(&tm_z, box, v0, i, gbase + col0, pol_first);
                     bulk_commit();
                   }
-                  // the box's sum over its 32 rows for request cr = lane & 15:
-                  // lane l reads rows 16 (l >> 4) .. + 15 of row cr of both
-                  // boxes with 128-bit loads (the swizzles spread each load over
-                  // all banks), and the two halves meet in one shuffle
-                  const int cr = lane & (kSub - 1), hf = lane >> 4;
-                  const float4* zrow4 = reinterpret_cast<const float4*>(box + cr * kUnit);
-                  const uint4* lrow4 = reinterpret_cast<const uint4*>(lobox + cr * kUnit);
-                  double us0 = 0.0, us1 = 0.0;
-#pragma unroll
-                  for (int qq = 0; qq < 2; ++qq) {
-                    const uint4 lv = lrow4[(2 * hf + qq) ^ ((cr >> 1) & 3)];
-                    const uint32_t lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                      const float4 zv = zrow4[(4 * hf + 2 * qq + h2) ^ (cr & 7)];
-                      const uint32_t a = lw[2 * h2], b = lw[2 * h2 + 1];
-                      double w0, w1, w2, w3;
-                      exp_fine2(f2(zv.x, zv.y), f2(__uint_as_float(a << 16), __uint_as_float(a & 0xffff0000u)), t16,
-                                &w0, &w1);
-                      exp_fine2(f2(zv.z, zv.w), f2(__uint_as_float(b << 16), __uint_as_float(b & 0xffff0000u)), t16,
-                                &w2, &w3);
-                      us0 += w0;
-                      us1 += w1;
-                      us0 += w2;
-                      us1 += w3;
-                    }
-                  }
-                  double us = us0 + us1;
-                  us += __shfl_xor_sync(0xffffffffu, us, 16);
+                  // the box's sum over its 32 rows for request cr = lane >> 1
+                  const int cr = lane >> 1;
+                  const double us = warp_transpose_sum16(wv, lane);
                   const int col = gbase + col0 + cr;
-                  if (lane < kSub && col0 + cr < nreal) {
+                  if ((lane & 1) == 0 && col0 + cr < nreal) {
                     acc[kk] += us;
                     p.unit_sum[static_cast<long long>(v0 / kUnit) * d.B + col] = us;
                   }
@@ -815,8 +774,8 @@ __global__ void __maxnreg__(96)
         // this warp's quadrant of the slice sums of group gr
 #pragma unroll
         for (int kk = 0; kk < kSubPerWarp; ++kk) {
-          const int col = (4 * kk + hh) * kSub + lane;
-          if (lane < kSub && kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[kk];
+          const int col = (4 * kk + hh) * kSub + (lane >> 1);
+          if ((lane & 1) == 0 && kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[kk];
         }
         release_pending(0);
         pending = gr;
@@ -935,7 +894,7 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
     cuuint32_t box[3] = {static_cast<cuuint32_t>(kUnit), 1, static_cast<cuuint32_t>(kSub)};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(ptr), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
   if (!enc3(&tm_base, a.base) || !enc3(&tm_z, a.z)) return cudaErrorInvalidValue;
