@@ -30,7 +30,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["bf16_to_f64", "softmax", "icdf", "markov_bias", "draft_step", "draft",
-           "survival", "schedule", "verify", "run_round", "calibrate"]
+           "survival", "schedule", "verify", "run_round", "calibrate", "round_to_bf16", "rnn_draft"]
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -325,3 +325,71 @@ def calibrate(conf, temps, verify_len, accepted, eta: float, t_min: float, t_max
         theta = theta - eta * g
         T[j - 1] = np.clip(1.0 / theta, t_min, t_max) if theta > 0 else t_max
     return T
+
+
+def round_to_bf16(x) -> np.ndarray:
+    """fp64 values rounded to the nearest bfloat16 (8 significant bits, ties to
+    even), returned as fp64. Direct from fp64 (no intermediate fp32 rounding):
+    for a normal x with 2^e <= |x| < 2^(e+1) the bf16 spacing is 2^(e-7), and
+    x / 2^(e-7) is exact in fp64, so rounding that quotient half-to-even and
+    scaling back is the correctly rounded value."""
+    x = np.asarray(x, np.float64)
+    out = np.zeros_like(x)
+    nz = (x != 0) & np.isfinite(x)
+    e = np.floor(np.log2(np.abs(x[nz])))
+    # guard against log2 landing one below an exact power of two
+    e = np.where(np.abs(x[nz]) >= 2.0 ** (e + 1), e + 1, e)
+    q = 2.0 ** (e - 7)
+    out[nz] = np.round(x[nz] / q) * q
+    out[~np.isfinite(x)] = x[~np.isfinite(x)]
+    return out
+
+
+def rnn_draft(base, A, W, Bf, anchor, u_draft, teacher=None, keep_z=True) -> dict:
+    """K-step draft with the RNN sequential head.
+
+    [QbitAI] section "a cheaper sequential module: the Markov head", last
+    paragraph, and [Essay] section "parallel drafts are fast ...": besides the
+    default Markov head (previous token only) the paper offers an RNN head that
+    tracks the prefix of the whole draft block; both are light sequential
+    modules that correct the parallel backbone's base logits left to right.
+    Reading (the pages give no equations): an Elman recurrence over the
+    drafted tokens with the Markov head's factors as input embedding and
+    output projection,
+        h_0 = 0,  h_i = tanh(A[t_{i-1}] + W h_{i-1}),  z_i = base_i + bf16(h_i) Bf,
+    t_0 the anchor, W [r,r] the recurrent weight; the state is rounded to
+    bfloat16 where it meets the bf16 projection, as the factors are. With
+    W = 0 this is the Markov head with factors bf16(tanh(A)).
+    Same outputs as draft() (teacher forcing included), plus "h" [B,K,r], the
+    fp64 states before rounding.
+    """
+    base = np.asarray(base)
+    B, K, V = base.shape
+    A64, Bf64 = factors_f64(A, Bf)
+    W64 = bf16_to_f64(W) if np.asarray(W).dtype == np.uint16 else np.asarray(W, np.float64)
+    r = A64.shape[1]
+    t_prev = np.asarray(anchor, np.int64)
+    h = np.zeros((B, r))
+    out = {k: [] for k in ("t", "q_tok", "lse", "margin", "z", "h")}
+    for i in range(K):
+        h = np.tanh(A64[t_prev] + h @ W64.T)
+        hb = round_to_bf16(h)
+        z = np.asarray(base[:, i], np.float64) + hb @ Bf64
+        zmax = z.max(axis=-1)
+        e = np.exp(z - zmax[:, None])
+        Wsum = e.sum(axis=-1)
+        q = e / Wsum[:, None]
+        t, margin = icdf(q, u_draft[:, i])
+        lse = zmax + np.log(Wsum)
+        chain = t if teacher is None else np.asarray(teacher[:, i], np.int64)
+        out["t"].append(t)
+        out["q_tok"].append(np.exp(z[np.arange(B), chain] - lse))
+        out["lse"].append(lse)
+        out["margin"].append(margin)
+        out["h"].append(h)
+        if keep_z:
+            out["z"].append(z)
+        t_prev = chain
+    res = {k: np.stack(v, axis=1) for k, v in out.items() if v}
+    res["chain"] = res["t"] if teacher is None else np.asarray(teacher, np.int64)
+    return res
