@@ -84,6 +84,27 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
                                   void* workspace, size_t ws_bytes, dspark_stream_t stream);
 
 /*
+ * The same draft with the RNN sequential head in place of the Markov head.
+ * [QbitAI] section "a cheaper sequential module: the Markov head", last
+ * paragraph, and [Essay] section "parallel drafts are fast ...": the paper
+ * offers an RNN head that tracks the prefix of the whole draft block (off by
+ * default). The pages give no equations; the head here is an Elman recurrence
+ * over the drafted tokens with the Markov factors as embedding and projection:
+ *   h_0 = 0,  h_i = tanh(A[t_{i-1},:] + W h_{i-1}),
+ *   z[b,i,:] = base_logits[b,i,:] + bf16(h_i) . Bf     (t_0 = anchor[b])
+ * with h in fp64 and rounded to bfloat16 (to nearest, ties to even) where it
+ * meets the bf16 projection. W [r,r] is bf16, row-major (W[k][m] multiplies
+ * h_{i-1}[m] into h_i[k]). Sampling, outputs and conventions are those of
+ * dspark_markov_draft. Needs bf16 factors, r a multiple of 64 up to 256 and
+ * V % 32 == 0 (the tensor-core kernel); other shapes return
+ * DSPARK_ERR_UNSUPPORTED.
+ */
+dspark_status dspark_rnn_draft(const float* base_logits, const void* A, const void* W, const void* Bf,
+                               dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft,
+                               int B, int K, int V, int32_t* draft_tokens, float* q_tok, double* lse_q,
+                               float* z, void* workspace, size_t ws_bytes, dspark_stream_t stream);
+
+/*
  * Confidence-scheduled verify lengths.
  * [QbitAI] section "variable-length drafts and hardware-aware scheduling"
  * (a confidence head scores each position's survival; a pre-measured

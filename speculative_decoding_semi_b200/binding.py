@@ -43,6 +43,8 @@ def _load() -> ctypes.CDLL:
     lib.dspark_workspace_init.restype = I
     lib.dspark_markov_draft.argtypes = [P, P, P, I, I, P, P, I, I, I, P, P, P, P, P, Z, S]
     lib.dspark_markov_draft.restype = I
+    lib.dspark_rnn_draft.argtypes = [P, P, P, P, I, I, P, P, I, I, I, P, P, P, P, P, Z, S]
+    lib.dspark_rnn_draft.restype = I
     lib.dspark_schedule.argtypes = [P, P, P, I, I, I, P, P, P, P, P, Z, S]
     lib.dspark_schedule.restype = I
     lib.dspark_verify.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, P, P, P, P, Z, S]
@@ -126,6 +128,23 @@ def dspark_markov_draft(base_logits, A, Bf, anchor, u_draft, draft_tokens, q_tok
         _ptr(lse_q, "lse_q", torch.float64, B * K), _ptr(z, "z", torch.float32, B * K * V),
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check("dspark_markov_draft", st)
+
+
+def dspark_rnn_draft(base_logits, A, W, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, z, workspace,
+                     stream=None) -> None:
+    """Draft with the RNN sequential head (W [r,r] bf16); bf16 factors only."""
+    B, K, V = base_logits.shape
+    r = A.shape[1]
+    if not (A.dtype == Bf.dtype == W.dtype == torch.bfloat16):
+        raise TypeError("the RNN head takes bf16 A, W and Bf")
+    st = lib.dspark_rnn_draft(
+        _ptr(base_logits, "base_logits", torch.float32), _ptr(A, "A", numel=V * r), _ptr(W, "W", numel=r * r),
+        _ptr(Bf, "Bf", numel=r * V), DSPARK_BF16, r, _ptr(anchor, "anchor", torch.int32, B),
+        _ptr(u_draft, "u_draft", torch.float32, B * K), B, K, V,
+        _ptr(draft_tokens, "draft_tokens", torch.int32, B * K), _ptr(q_tok, "q_tok", torch.float32, B * K),
+        _ptr(lse_q, "lse_q", torch.float64, B * K), _ptr(z, "z", torch.float32, B * K * V),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("dspark_rnn_draft", st)
 
 
 def dspark_schedule(conf_logits, temps, profile_ms, verify_len, survival, row_start, n_tokens, workspace,

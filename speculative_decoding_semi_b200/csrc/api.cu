@@ -48,16 +48,21 @@ dspark_status dspark_workspace_init(void* workspace, size_t ws_bytes, dspark_str
   return from_cuda(cudaMemsetAsync(workspace, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-dspark_status dspark_markov_draft(const float* base_logits, const void* A, const void* Bf,
-                                  dspark_dtype factor_dtype, int r, const int32_t* anchor,
-                                  const float* u_draft, int B, int K, int V, int32_t* draft_tokens,
-                                  float* q_tok, double* lse_q, float* z, void* workspace,
-                                  size_t ws_bytes, dspark_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The Markov head (W == nullptr) or the RNN head (W = its recurrent weight).
+dspark_status draft_call(const float* base_logits, const void* A, const void* W, const void* Bf,
+                         dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft, int B, int K,
+                         int V, int32_t* draft_tokens, float* q_tok, double* lse_q, float* z, void* workspace,
+                         size_t ws_bytes, dspark_stream_t stream) {
   if (!sizes_ok(B, K, V) || r < 1 || r > kMaxR) return DSPARK_ERR_INVALID_ARG;
   if (factor_dtype != DSPARK_F32 && factor_dtype != DSPARK_BF16) return DSPARK_ERR_INVALID_ARG;
   const void* ptrs[] = {base_logits, A, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, z, workspace};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
+  if (W != nullptr && !aligned16(W)) return DSPARK_ERR_INVALID_ARG;
   if (ws_bytes < dspark_workspace_bytes(B, K, V, r)) return DSPARK_ERR_INVALID_ARG;
   if (2u * K * sizeof(unsigned) > kSyncBytes) return DSPARK_ERR_INVALID_ARG;
 
@@ -70,6 +75,7 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
   a.base = base_logits;
   a.A = A;
   a.Bf = Bf;
+  a.W = W;
   a.bf16 = factor_dtype == DSPARK_BF16;
   a.r = r;
   a.anchor = anchor;
@@ -85,7 +91,9 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
   a.sync = reinterpret_cast<unsigned*>(ws + kSyncOffset);
   // bf16 factors with r % 64 == 0 (r <= 256) and V % 32 == 0 take the
   // tensor-core kernel; other shapes and fp32 factors the CUDA-core kernel
+  // (which has the Markov head only)
   const bool tc = draft_tc_supported(a);
+  if (W != nullptr && !tc) return DSPARK_ERR_UNSUPPORTED;
   const int G = tc ? draft_tc_grid(V, sms) : draft_grid_size(V, sms);
   char* scratch = ws + kScratchOffset + schedule_region(B, K) + verify_region(B, K, V);
   const size_t gmax = std::min<size_t>(kMaxGrid, V / 8);
@@ -97,6 +105,28 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
   cudaError_t e = cudaMemsetAsync(a.sync, 0, kSyncBytes, s);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   return from_cuda(tc ? launch_draft_tc(a, G, a.sync, extra, s) : launch_draft_generic(a, G, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+dspark_status dspark_markov_draft(const float* base_logits, const void* A, const void* Bf,
+                                  dspark_dtype factor_dtype, int r, const int32_t* anchor,
+                                  const float* u_draft, int B, int K, int V, int32_t* draft_tokens,
+                                  float* q_tok, double* lse_q, float* z, void* workspace,
+                                  size_t ws_bytes, dspark_stream_t stream) {
+  return draft_call(base_logits, A, nullptr, Bf, factor_dtype, r, anchor, u_draft, B, K, V, draft_tokens, q_tok,
+                    lse_q, z, workspace, ws_bytes, stream);
+}
+
+dspark_status dspark_rnn_draft(const float* base_logits, const void* A, const void* W, const void* Bf,
+                               dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft, int B,
+                               int K, int V, int32_t* draft_tokens, float* q_tok, double* lse_q, float* z,
+                               void* workspace, size_t ws_bytes, dspark_stream_t stream) {
+  if (W == nullptr) return DSPARK_ERR_INVALID_ARG;
+  return draft_call(base_logits, A, W, Bf, factor_dtype, r, anchor, u_draft, B, K, V, draft_tokens, q_tok, lse_q, z,
+                    workspace, ws_bytes, stream);
 }
 
 dspark_status dspark_schedule(const float* conf_logits, const float* temps, const float* profile_ms,

@@ -95,6 +95,8 @@ struct TcParams {
   int nbs;              // base/z ring slots per epilogue warp
   int image_stride;     // bytes per group in the operand image (and in shared memory)
   double* unit_sum;     // [V/32][B] sums of exp(z) over each 32-row unit, this position
+  double* hstate;       // [B][r] RNN head: state h_i of each request (fp64)
+  double* ustate;       // [B][r] RNN head: W h_i, formed while position i streams
 };
 
 struct Layout {
@@ -381,6 +383,98 @@ __device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t,
   }
 }
 
+// ------------------------------------------------------------- RNN head
+// QbitAI article, section "a cheaper sequential module: the Markov head",
+// last paragraph (and the 10100.com essay, section "parallel drafts are fast
+// ..."): an optional RNN head tracks the prefix of the whole draft block. Here
+// h_0 = 0, h_i = tanh(A[t_{i-1}] + W h_{i-1}), and the operand row of request
+// b at position i is bf16(h_i) instead of A[t_{i-1}]; the state stays in fp64.
+// Lane l owns the state's elements 8l .. 8l+7 (one 16-byte chunk of the
+// operand row), for r/8 <= 32 lanes.
+
+// fp64 -> bf16 bits, round to nearest even directly from the fp64 value
+// (no fp32 step); values below bf16's normal range round on its subnormal
+// grid. For finite inputs of magnitude < 2^128.
+__device__ __forceinline__ uint16_t f64_to_bf16_bits(double x) {
+  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(x));
+  const unsigned sign = static_cast<unsigned>(u >> 63) << 15;
+  const double ax = fabs(x);
+  if (ax < 1.1754943508222875e-38) {  // 2^-126: subnormal grid 2^-133
+    const double m = rint(ax * 1.0889035741470030e+40);  // * 2^133
+    return static_cast<uint16_t>(sign | static_cast<unsigned>(m));
+  }
+  const int e = static_cast<int>((u >> 52) & 0x7FF) - 1023 + 127;
+  unsigned long long m = u & ((1ull << 52) - 1);
+  const unsigned long long low = m & ((1ull << 45) - 1), half = 1ull << 44;
+  m >>= 45;
+  unsigned bits = (static_cast<unsigned>(e) << 7) | static_cast<unsigned>(m);
+  if (low > half || (low == half && (m & 1))) ++bits;  // a carry moves into the exponent
+  return static_cast<uint16_t>(sign | bits);
+}
+
+// U = W h for request b (one warp, fp64): lane l forms U[8l .. 8l+7]; the
+// state's chunks are passed between lanes by shuffles.
+__device__ __noinline__ void rnn_matvec(const TcParams& p, int b, int lane) {
+  const int r = p.d.r, nch = r / 8;
+  const uint16_t* W = static_cast<const uint16_t*>(p.d.W);
+  const double* h = p.hstate + static_cast<long long>(b) * r;
+  double hl[8], u[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    hl[e] = lane < nch ? h[8 * lane + e] : 0.0;
+    u[e] = 0.0;
+  }
+  for (int c = 0; c < nch; ++c) {
+    double hm[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hm[e] = __shfl_sync(0xffffffffu, hl[e], c);
+    if (lane < nch) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(W + static_cast<long long>(8 * lane + k) * r + 8 * c));
+        const uint32_t wp[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          u[k] = fma(static_cast<double>(__uint_as_float(wp[e] << 16)), hm[2 * e], u[k]);
+          u[k] = fma(static_cast<double>(__uint_as_float(wp[e] & 0xffff0000u)), hm[2 * e + 1], u[k]);
+        }
+      }
+    }
+  }
+  if (lane < nch) {
+    double* us = p.ustate + static_cast<long long>(b) * r + 8 * lane;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) us[k] = u[k];
+  }
+}
+
+// h = tanh(A[t] + U) (U = W h_prev, or 0 at the first position) for request
+// b: stored as the new state and written, rounded to bf16, as b's operand row.
+__device__ __noinline__ void rnn_step(const TcParams& p, int b, int t, bool first, int lane) {
+  const int r = p.d.r, nch = r / 8;
+  if (lane >= nch) return;
+  const int gr = b / p.gsize, n = b - gr * p.gsize;
+  const int N = round16(group_real(p, gr));
+  const uint4 av = __ldg(reinterpret_cast<const uint4*>(p.d.A) + static_cast<long long>(t) * nch + lane);
+  const uint32_t ap[4] = {av.x, av.y, av.z, av.w};
+  double* hs = p.hstate + static_cast<long long>(b) * r + 8 * lane;
+  const double* us = p.ustate + static_cast<long long>(b) * r + 8 * lane;
+  uint32_t out[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const double u0 = first ? 0.0 : us[2 * e], u1 = first ? 0.0 : us[2 * e + 1];
+    const double h0 = tanh(static_cast<double>(__uint_as_float(ap[e] << 16)) + u0);
+    const double h1 = tanh(static_cast<double>(__uint_as_float(ap[e] & 0xffff0000u)) + u1);
+    hs[2 * e] = h0;
+    hs[2 * e + 1] = h1;
+    out[e] = static_cast<uint32_t>(f64_to_bf16_bits(h0)) | (static_cast<uint32_t>(f64_to_bf16_bits(h1)) << 16);
+  }
+  uint8_t* img = p.image + static_cast<long long>(gr) * p.image_stride;
+  const int kb = lane >> 3, c = lane & 7;
+  *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
+      make_uint4(out[0], out[1], out[2], out[3]);
+}
+
 // One warp: every lane waits for *ctr >= target (bounded), so the warp stays
 // converged for the collective code that follows. Each lane's own acquire load
 // of the counter orders its later reads; no further fence is needed.
@@ -392,6 +486,7 @@ __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned 
 }
 
 // 19 warps: five share a 16K-register SM sub-partition, so at most 96 registers each
+template <bool kRnn>
 __global__ void __maxnreg__(96)
     draft_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_bf,
                     const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_z) {
@@ -564,7 +659,10 @@ __global__ void __maxnreg__(96)
     // ------------------------------------------------------------ selector
     bool ok = true;
     // position 0's operand: the anchors' rows, and zeros in padded rows
-    for (int b = g; b < d.B; b += G) write_image_row(p, b, previous_token(d, b, 0), lane);
+    for (int b = g; b < d.B; b += G) {
+      if (kRnn) rnn_step(p, b, previous_token(d, b, 0), true, lane);
+      else write_image_row(p, b, previous_token(d, b, 0), lane);
+    }
     if (g == 0) {
       for (int gr = 0; gr < p.ngroups; ++gr) {
         const int nreal = group_real(p, gr), N = round16(nreal);
@@ -595,6 +693,9 @@ __global__ void __maxnreg__(96)
     for (int i = 0; ok && i < d.K; ++i) {
       for (int gr = 0; ok && gr < p.ngroups; ++gr) {
         const int gbase = gr * p.gsize, nreal = group_real(p, gr);
+        // RNN head: W h_i of this CTA's requests, while position i streams
+        if (kRnn && i + 1 < d.K)
+          for (int b = gbase + ((g - gbase) % G + G) % G; b < gbase + nreal; b += G) rnn_matvec(p, b, lane);
         if (!mbar_wait(bars.step_done(gr), i & 1, s_abort, d.err, 0x500u)) {
           ok = false;
           break;
@@ -620,7 +721,10 @@ __global__ void __maxnreg__(96)
           if (!ok) break;
           for (int b = first; b < gbase + nreal; b += G) {
             const int t = select_warp(p, b, i, G, lane, t16);
-            if (i + 1 < d.K) write_image_row(p, b, t, lane);
+            if (i + 1 < d.K) {
+              if (kRnn) rnn_step(p, b, t, false, lane);
+              else write_image_row(p, b, t, lane);
+            }
             ++mine;
           }
         }
@@ -837,8 +941,11 @@ size_t image_bytes(int B, int r) {
   return align_up(ngroups * gs * r * 2, 256);
 }
 
+size_t unit_sum_bytes(int B, int V) { return align_up(static_cast<size_t>(V / kUnit) * B * sizeof(double), 256); }
+size_t rnn_state_bytes(int B, int r) { return align_up(static_cast<size_t>(B) * r * sizeof(double), 256); }
+
 size_t draft_tc_extra_bytes(int B, int V, int r) {
-  return image_bytes(B, r) + align_up(static_cast<size_t>(V / kUnit) * B * sizeof(double), 256);
+  return image_bytes(B, r) + unit_sum_bytes(B, V) + 2 * rnn_state_bytes(B, r);
 }
 
 cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cudaStream_t stream) {
@@ -856,6 +963,8 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
   p.image_stride = p.gsize * a.r * 2;
   p.image = reinterpret_cast<uint8_t*>(extra);
   p.unit_sum = reinterpret_cast<double*>(extra + image_bytes(a.B, a.r));
+  p.hstate = reinterpret_cast<double*>(extra + image_bytes(a.B, a.r) + unit_sum_bytes(a.B, a.V));
+  p.ustate = p.hstate + rnn_state_bytes(a.B, a.r) / sizeof(double);
   p.sync_part = sync;
   p.sync_tok = sync + a.K * p.ngroups;
   int dev = 0, max_smem = 0;
@@ -899,18 +1008,19 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
   };
   if (!enc3(&tm_base, a.base) || !enc3(&tm_z, a.z)) return cudaErrorInvalidValue;
 
-  cudaError_t e = cudaFuncSetAttribute(draft_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  // the Markov head's kernel carries no code of the RNN head
+  const void* fn = a.W != nullptr ? reinterpret_cast<const void*>(&draft_tc_kernel<true>)
+                                  : reinterpret_cast<const void*>(&draft_tc_kernel<false>);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, draft_tc_kernel, kThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
   if (e != cudaSuccess) return e;
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (per_sm < 1 || G > per_sm * sms) return cudaErrorCooperativeLaunchTooLarge;
   void* args[] = {&p, &tm_bf, &tm_base, &tm_z};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(draft_tc_kernel), dim3(G), dim3(kThreads), args,
-                                     smem, stream);
+  return cudaLaunchCooperativeKernel(fn, dim3(G), dim3(kThreads), args, smem, stream);
 }
 
 }  // namespace dspark

@@ -26,6 +26,7 @@ struct DraftArgs {
   unsigned* sync;   // 2*K counters
   float* part_m;    // [B][G]
   double* part_S;   // [B][G]
+  const void* W;    // RNN head's recurrent weight [r,r] (bf16), or null for the Markov head
 };
 
 struct VerifyArgs {

@@ -8,8 +8,7 @@
 // time + verify time) / accepted tokens. Section "online drafter
 // calibration": sequential temperature scaling of the confidence.
 //
-// Up to 1024 items, one kernel (one CTA, arrays in shared memory) does both
-// steps below; larger batches use two kernels:
+// Two kernels:
 //   rank  : every CTA recomputes the survival products P[b,j] in fp64 (cheap,
 //           bit-identical in every CTA) and ranks its items among all B*K by
 //           (P desc, j asc, b asc). Request b's items are a non-increasing
@@ -35,6 +34,10 @@ __device__ __forceinline__ bool precedes(double Pa, int ja, int ba, double Pb, i
 
 __global__ void __launch_bounds__(ST) schedule_rank_kernel(ScheduleArgs a, int tpi) {
   extern __shared__ double P[];  // [B*K]
+  // launched early (programmatic dependent launch): the previous kernel's
+  // writes are visible after the wait; the final kernel may launch meanwhile
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int B = a.B, K = a.K, N = B * K;
   for (int b = threadIdx.x; b < B; b += ST) {
     double prod = 1.0;
@@ -76,22 +79,20 @@ __global__ void __launch_bounds__(ST) schedule_rank_kernel(ScheduleArgs a, int t
   }
 }
 
-// The final step (one CTA of FT threads, all of which call): prefix sums of
-// the ranked values, the smallest maximiser m*, lengths and row offsets.
-// `sorted` and `rank` are the rank step's outputs (global or shared memory).
-__device__ __forceinline__ void schedule_finish(const ScheduleArgs& a, const double* sorted, const int32_t* rank) {
+__global__ void __launch_bounds__(FT) schedule_final_kernel(ScheduleArgs a) {
   __shared__ double redd[33];
   __shared__ double s_best[32];
   __shared__ int s_bestm[32];
   __shared__ int s_mstar;
   __shared__ long long redl[33];
   const int B = a.B, K = a.K, N = B * K, tid = threadIdx.x;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the rank kernel's results
   const int M = min(N, a.n_prof - B);
   // prefix sums S_m over the ranked values, m = 1..N
   const int per = (N + FT - 1) / FT;
   const int lo = min(N, tid * per), hi = min(N, lo + per);
   double local = 0.0;
-  for (int k = lo; k < hi; ++k) local += sorted[k];
+  for (int k = lo; k < hi; ++k) local += a.sorted_P[k];
   double total;
   const double ex = block_exclusive_scan<FT>(local, redd, &total);
   // objective (B + S_m) / T(B + m); T(n) = profile[n - 1]
@@ -103,7 +104,7 @@ __device__ __forceinline__ void schedule_finish(const ScheduleArgs& a, const dou
   }
   double S = ex;
   for (int k = lo; k < hi; ++k) {
-    S += sorted[k];
+    S += a.sorted_P[k];
     const int m = k + 1;
     if (m > M) break;
     const double obj = (static_cast<double>(B) + S) / static_cast<double>(a.profile[B + m - 1]);
@@ -147,7 +148,7 @@ __device__ __forceinline__ void schedule_finish(const ScheduleArgs& a, const dou
   long long lcount = 0;
   for (int b = b_lo; b < b_hi; ++b) {
     int L = 0;
-    for (int j = 0; j < K; ++j) L += (rank[b * K + j] < mstar) ? 1 : 0;
+    for (int j = 0; j < K; ++j) L += (a.rank[b * K + j] < mstar) ? 1 : 0;
     a.verify_len[b] = L;
     lcount += L + 1;
   }
@@ -181,57 +182,6 @@ __device__ __forceinline__ void schedule_finish(const ScheduleArgs& a, const dou
   }
 }
 
-__global__ void __launch_bounds__(FT) schedule_final_kernel(ScheduleArgs a) { schedule_finish(a, a.sorted_P, a.rank); }
-
-// Small batches (B*K <= kSingleMax): the whole schedule in one CTA, its
-// arrays in shared memory; the ranking is the rank kernel's, with tpi threads
-// per item.
-constexpr int kSingleMax = 1024;
-
-__global__ void __launch_bounds__(FT) schedule_single_kernel(ScheduleArgs a, int tpi) {
-  __shared__ double P[kSingleMax];
-  __shared__ double sorted[kSingleMax];
-  __shared__ int32_t rank[kSingleMax];
-  const int B = a.B, K = a.K, N = B * K;
-  for (int b = threadIdx.x; b < B; b += FT) {
-    double prod = 1.0;
-    for (int j = 0; j < K; ++j) {
-      const double x = static_cast<double>(a.conf[b * K + j]) / static_cast<double>(a.temps[j]);
-      const double s = 1.0 / (1.0 + exp(-x));
-      prod = __dmul_rn(prod, s);
-      P[b * K + j] = prod;
-      a.survival[b * K + j] = static_cast<float>(prod);
-    }
-  }
-  __syncthreads();
-  const int lane = threadIdx.x % tpi;
-  for (int base = 0; base < N; base += FT / tpi) {
-    const int item = base + threadIdx.x / tpi;
-    const bool valid = item < N;
-    const int b = valid ? item / K : 0, j = valid ? item - b * K : 0;
-    const double p = valid ? P[item] : 0.0;
-    int cnt = 0;
-    if (valid) {
-      for (int bp = lane; bp < B; bp += tpi) {
-        int lo = 0, hi = K;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (precedes(P[bp * K + mid], mid, bp, p, j, b)) lo = mid + 1;
-          else hi = mid;
-        }
-        cnt += lo;
-      }
-    }
-    for (int o = tpi / 2; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o, tpi);
-    if (valid && lane == 0) {
-      rank[item] = cnt;
-      sorted[cnt] = p;
-    }
-  }
-  __syncthreads();
-  schedule_finish(a, sorted, rank);
-}
-
 }  // namespace
 
 size_t schedule_scratch_bytes(int B, int K) {
@@ -245,19 +195,42 @@ cudaError_t launch_schedule(ScheduleArgs a, char* scratch, cudaStream_t stream) 
   a.sorted_P = reinterpret_cast<double*>(scratch + align_up(N * sizeof(int32_t), 256));
   int tpi = 1;
   while (tpi < 32 && tpi * 8 < a.B) tpi <<= 1;
-  if (N <= static_cast<size_t>(kSingleMax)) {
-    schedule_single_kernel<<<1, FT, 0, stream>>>(a, tpi);
-    return cudaGetLastError();
-  }
   const size_t smem = N * sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(schedule_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const long long threads = static_cast<long long>(N) * tpi;
   const int grid = static_cast<int>(std::max<long long>(1, (threads + ST - 1) / ST));
-  schedule_rank_kernel<<<grid, ST, smem, stream>>>(a, tpi);
-  schedule_final_kernel<<<1, FT, 0, stream>>>(a);
-  return cudaGetLastError();
+  // both kernels are launched with programmatic stream serialisation, so that
+  // each one's launch overlaps the kernel before it; each waits (griddepcontrol)
+  // for its predecessor's results before reading anything
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(ST);
+  cfg.dynamicSmemBytes = smem;
+  e = cudaLaunchKernelEx(&cfg, schedule_rank_kernel, a, tpi);
+  if (e == cudaErrorNotSupported) {  // without the early launch
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, schedule_rank_kernel, a, tpi);
+  }
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(FT);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, schedule_final_kernel, a);
+  if (e == cudaErrorNotSupported) {
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, schedule_final_kernel, a);
+  }
+  return e;
 }
 
 }  // namespace dspark

@@ -66,7 +66,6 @@ constexpr int kStageBytes = kRowItem * 4;
 constexpr int kStages = 6;
 constexpr int kPlanThreads = 1024;
 constexpr int kRegSeg = 8;                // segment values per lane held in registers (nseg <= 256)
-constexpr int kRegWeight = 12;            // segment weights per lane held in registers
 constexpr double kSumLo = 1e-20, kSumHi = 1e30;
 constexpr float kLog2e = 1.44269504088896340736f;  // log2(e)
 constexpr double kLog2eD = 1.44269504088896340736;
@@ -186,8 +185,10 @@ __device__ int block_exscan_int(int v, int* total, int* red) {
 
 __global__ void __launch_bounds__(kPlanThreads) verify_plan_kernel(Params p) {
   __shared__ int red[33];
-  // the main kernel may start its prologue now; it waits for this grid's
-  // results before reading them
+  // launched early (programmatic dependent launch): the previous kernel's
+  // writes (verify lengths, drafts) are visible after the wait; the main
+  // kernel may start its prologue now and waits for this grid's results
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const VerifyArgs& a = p.a;
   int carry = 0;
@@ -900,9 +901,24 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(kStages) * kStageBytes + sizeof(Smem);
   e = cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  verify_plan_kernel<<<1, kPlanThreads, 0, stream>>>(P);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  {
+    cudaLaunchAttribute pattr[1];
+    pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pattr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t pcfg{};
+    pcfg.gridDim = dim3(1);
+    pcfg.blockDim = dim3(kPlanThreads);
+    pcfg.stream = stream;
+    pcfg.attrs = pattr;
+    pcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&pcfg, verify_plan_kernel, P);
+    if (e == cudaErrorNotSupported) {  // without the early launch
+      (void)cudaGetLastError();
+      pcfg.numAttrs = 0;
+      e = cudaLaunchKernelEx(&pcfg, verify_plan_kernel, P);
+    }
+    if (e != cudaSuccess) return e;
+  }
   const long long rows = static_cast<long long>(a.B) * (a.K + 1);
   const long long units = std::max(rows * P.ngrp, (rows + kWarps - 1) / kWarps);
   const int G = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, units)));

@@ -12,8 +12,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from .binding import (dspark_advance_anchor, dspark_calibrate, dspark_markov_draft, dspark_schedule, dspark_verify,
-                      dspark_workspace_bytes, dspark_workspace_init)
+from .binding import (dspark_advance_anchor, dspark_calibrate, dspark_markov_draft, dspark_rnn_draft, dspark_schedule,
+                      dspark_verify, dspark_workspace_bytes, dspark_workspace_init)
 
 
 def to_device(inputs: dict, device="cuda") -> dict:
@@ -22,7 +22,7 @@ def to_device(inputs: dict, device="cuda") -> dict:
     for k, v in inputs.items():
         if not isinstance(v, np.ndarray):
             continue
-        if k in ("A", "Bf") and v.dtype == np.uint16:
+        if k in ("A", "Bf", "W") and v.dtype == np.uint16:
             out[k] = torch.from_numpy(v.view(np.int16)).to(device).view(torch.bfloat16)
         else:
             out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device)
@@ -53,8 +53,13 @@ class RoundBuffers:
 
 
 def draft(d: dict, bufs: RoundBuffers, stream=None):
-    dspark_markov_draft(d["base"], d["A"], d["Bf"], d["anchor"], d["u_draft"], bufs.draft_tokens, bufs.q_tok,
-                        bufs.lse_q, bufs.z, bufs.workspace, stream)
+    """The Markov head, or the RNN head when d holds its recurrent weight "W"."""
+    if d.get("W") is not None:
+        dspark_rnn_draft(d["base"], d["A"], d["W"], d["Bf"], d["anchor"], d["u_draft"], bufs.draft_tokens, bufs.q_tok,
+                         bufs.lse_q, bufs.z, bufs.workspace, stream)
+    else:
+        dspark_markov_draft(d["base"], d["A"], d["Bf"], d["anchor"], d["u_draft"], bufs.draft_tokens, bufs.q_tok,
+                            bufs.lse_q, bufs.z, bufs.workspace, stream)
 
 
 def schedule(d: dict, bufs: RoundBuffers, stream=None):

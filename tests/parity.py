@@ -68,10 +68,15 @@ def within_rate(excused: int, decisions: int) -> bool:
 
 
 def compare_draft(inp, gpu, requests, tally: Tally, check_z=True):
-    """gpu: dict of numpy outputs for the sampled `requests` (tokens, q_tok, lse_q, z)."""
+    """gpu: dict of numpy outputs for the sampled `requests` (tokens, q_tok, lse_q, z).
+    With inp["W"] (the RNN head's recurrent weight) the oracle is rnn_draft."""
     base = inp["base"][requests]
-    d = oracle.draft(base, inp["A"], inp["Bf"], inp["anchor"][requests], inp["u_draft"][requests],
-                     teacher=gpu["tokens"].astype(np.int64), keep_z=True)
+    if inp.get("W") is not None:
+        d = oracle.rnn_draft(base, inp["A"], inp["W"], inp["Bf"], inp["anchor"][requests], inp["u_draft"][requests],
+                             teacher=gpu["tokens"].astype(np.int64), keep_z=True)
+    else:
+        d = oracle.draft(base, inp["A"], inp["Bf"], inp["anchor"][requests], inp["u_draft"][requests],
+                         teacher=gpu["tokens"].astype(np.int64), keep_z=True)
     mism = d["t"] != gpu["tokens"]
     small = d["margin"] < MARGIN
     tally.flagged += int(small.sum())
