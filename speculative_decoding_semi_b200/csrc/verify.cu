@@ -21,11 +21,11 @@
 //                 logit at the drafted token;
 //     2 row stats one warp per row: (max, sum) from the segment partials and
 //                 the accept test u * q(t) < p(t) of the row's draft;
-//     3 decide    one warp per request: the first rejection; with none, the
-//                 bonus token is drawn at once; else the request joins the
-//                 list of residual passes;
+//     3 decide    one warp per request: the first rejection; the request
+//                 joins the list of bonus draws (none) or of residual passes;
 //     4 residual  the rejected rows and their z rows stream through the same
-//                 ring: sums of max(0, p - q) over 512-wide segments;
+//                 ring: sums of max(0, p - q) over 512-wide segments; the
+//                 warps outside the stream make the bonus draws meanwhile;
 //     5 resample  one warp per listed request draws the resampled token.
 // The barriers fall between streaming phases, when no copy is in flight: a
 // gpu-scope fence on an SM with bulk copies in flight waits for them to land,
@@ -71,7 +71,8 @@ constexpr float kLog2e = 1.44269504088896340736f;  // log2(e)
 constexpr double kLog2eD = 1.44269504088896340736;
 
 enum : int { kItemRow = 0, kItemRes = 1, kItemExit = 2 };
-enum : int { kCtlRows = 0, kCtlListed = 1, kCtlBar = 2 };  // kCtlBar..kCtlBar+3: barrier counters
+// kCtlBar..kCtlBar+3: barrier counters
+enum : int { kCtlRows = 0, kCtlListed = 1, kCtlBar = 2, kCtlBonus = 6, kCtlCount = 8 };
 
 // One target row of the compact numbering.
 struct RowInfo {
@@ -108,6 +109,7 @@ struct Ws {
   ResDec* dec;       // [B]
   float2* resfac;    // [B][nseg] residual (shift, p factor) per 1024-segment
   int* list;         // [B] requests with a residual pass
+  int* blist;        // [B] requests whose drafts were all accepted (bonus draw)
   double* seg_w;     // [B][nrseg] residual segment sums
 };
 
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(kPlanThreads) verify_plan_kernel(Params p) {
     }
     carry += total;
   }
-  if (threadIdx.x < 8) p.w.ctl[threadIdx.x] = threadIdx.x == kCtlRows ? static_cast<unsigned>(carry) : 0u;
+  if (threadIdx.x < kCtlCount) p.w.ctl[threadIdx.x] = threadIdx.x == kCtlRows ? static_cast<unsigned>(carry) : 0u;
 }
 
 // ------------------------------------------------------ warp-level helpers
@@ -476,9 +478,11 @@ __device__ void write_output(const Params& P, int b, int acc, int tok, int lane)
   }
 }
 
-// Phase 3, one warp: request b's first rejection; the bonus draw, or the
-// residual pass's inputs and a place in the list.
-__device__ __noinline__ void decide(const Params& P, int b, int lane) {
+// Phase 3, one warp: request b's first rejection; a place in the list of
+// bonus draws, or the residual pass's inputs and a place in its list.
+// With `warm` set it writes nothing: it runs once during phase 1 to load its
+// code into the SM's instruction cache ahead of phase 3.
+__device__ __noinline__ void decide(const Params& P, int b, int lane, bool warm = false) {
   const VerifyArgs& a = P.a;
   const int r0 = P.w.rowbase[b];
   if (r0 < 0) return;  // invalid request (recorded by the plan kernel)
@@ -489,8 +493,9 @@ __device__ __noinline__ void decide(const Params& P, int b, int lane) {
   const int acc = m ? __ffs(m) - 1 : L;
   const int R = r0 + acc;
   if (acc == L) {
-    const int tok = sample_p(P, R, a.u_resample[b], lane);
-    write_output(P, b, L, tok, lane);
+    // the bonus draw is made during the residual pass, by the warps that
+    // pass leaves idle
+    if (lane == 0 && !warm) P.w.blist[atomicAdd(P.w.ctl + kCtlBonus, 1u)] = b;
     return;
   }
   const double M = __ldcg(&P.w.rstat[R].M), W = __ldcg(&P.w.rstat[R].W);
@@ -506,7 +511,8 @@ __device__ __noinline__ void decide(const Params& P, int b, int lane) {
 #pragma unroll
     for (int j = 0; j < kRegSeg; ++j) {
       const int q = q0 + lane + 32 * j;
-      if (q < P.nseg) rf[q] = res_factor(mv[j], M, W);
+      const float2 f = res_factor(mv[j], M, W);
+      if (q < P.nseg && !warm) rf[q] = f;
     }
   }
   if (lane == 0) {
@@ -515,8 +521,10 @@ __device__ __noinline__ void decide(const Params& P, int b, int lane) {
     d.R = R;
     d.row = P.w.rowinfo[R].row;
     q_factor(a.lse_q[static_cast<long long>(b) * a.K + acc], &d.mq, &d.fq);
-    P.w.dec[b] = d;
-    P.w.list[atomicAdd(P.w.ctl + kCtlListed, 1u)] = b;
+    if (!warm) {
+      P.w.dec[b] = d;
+      P.w.list[atomicAdd(P.w.ctl + kCtlListed, 1u)] = b;
+    }
   }
 }
 
@@ -775,7 +783,10 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
       d.row = P.w.rowinfo[0].row;
       r = residual_token(P, 0, d, 0.5f, lane, true);
     }
-    if (warp == kProdWarp + 3) row_stats(P, 0, lane);  // rewritten in phase 2
+    if (warp == kProdWarp + 3) {
+      row_stats(P, 0, lane);  // rewritten in phase 2
+      decide(P, 0, lane, true);
+    }
     if (lane == 0) s_sink = r;
   }
   ok = __syncthreads_and(ok) && grid_barrier(P, 0, &s_flag);
@@ -785,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
     for (int R = gw; R < n_rows; R += NW) row_stats(P, R, lane);
   ok = ok && grid_barrier(P, 1, &s_flag);
 
-  // ---- phase 3: decisions, bonus draws, residual list
+  // ---- phase 3: decisions; the bonus and residual lists
   if (ok)
     for (int b = gw; b < a.B; b += NW) decide(P, b, lane);
   ok = ok && grid_barrier(P, 2, &s_flag);
@@ -824,6 +835,17 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
                          pol_first);
         },
         [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_res(P, ds, stage, empty, w, lane); });
+    // meanwhile the warps outside the stream make the bonus draws
+    if (warp > kProdWarp) {
+      const int n_bonus = static_cast<int>(__ldcg(P.w.ctl + kCtlBonus));
+      const int nsw = (kWarps - kProdWarp - 1) * G;
+      for (int e = (warp - kProdWarp - 1) * G + c; e < n_bonus; e += nsw) {
+        const int b = __ldcg(P.w.blist + e);
+        const int L = a.verify_len[b];
+        const int tok = sample_p(P, P.w.rowbase[b] + L, a.u_resample[b], lane);
+        write_output(P, b, L, tok, lane);
+      }
+    }
     ok = __syncthreads_and(ok) && grid_barrier(P, 3, &s_flag);
   }
 
@@ -839,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
 }
 
 struct Layout {
-  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, seg_w, total;
+  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, blist, seg_w, total;
 };
 
 Layout verify_layout(int B, int K, int V) {
@@ -854,7 +876,7 @@ Layout verify_layout(int B, int K, int V) {
   };
   L.rowinfo = take(rows * sizeof(RowInfo));
   L.rowbase = take(nb * sizeof(int));
-  L.ctl = take(8 * sizeof(unsigned));
+  L.ctl = take(kCtlCount * sizeof(unsigned));
   L.part_m = take(rows * nseg * sizeof(float));
   L.part_S = take(rows * nseg * sizeof(double));
   L.x_tok = take(rows * sizeof(float));
@@ -863,6 +885,7 @@ Layout verify_layout(int B, int K, int V) {
   L.dec = take(nb * sizeof(ResDec));
   L.resfac = take(nb * nseg * sizeof(float2));
   L.list = take(nb * sizeof(int));
+  L.blist = take(nb * sizeof(int));
   L.seg_w = take(nb * nrseg * sizeof(double));
   L.total = off;
   return L;
@@ -891,6 +914,7 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
   P.w.dec = reinterpret_cast<ResDec*>(region + L.dec);
   P.w.resfac = reinterpret_cast<float2*>(region + L.resfac);
   P.w.list = reinterpret_cast<int*>(region + L.list);
+  P.w.blist = reinterpret_cast<int*>(region + L.blist);
   P.w.seg_w = reinterpret_cast<double*>(region + L.seg_w);
 
   int dev = 0, sms = 148;
