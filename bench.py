@@ -344,6 +344,7 @@ def run_gpu(args):
         "data": "synthetic", "config": config_of(w),
         "tokens_per_s": value * float(n_out.sum()),
         "stages_ms_median": {"draft": med(t_draft), "schedule": med(t_sched), "verify": med(t_ver)},
+        "draft_us_per_position": 1000.0 * med(t_draft) / K,
         "round_ms": {"median": med(t_round), "p10": float(np.percentile(t_round, 10)),
                      "p90": float(np.percentile(t_round, 90))},
         "roofline": {"bound": "hbm", "kernel": "dspark_markov_draft", "achieved": draft_gbs,
