@@ -75,7 +75,8 @@ dspark_status dspark_workspace_init(void* workspace, size_t ws_bytes, dspark_str
  * Outputs: draft_tokens [B,K] i32; q_tok [B,K] f32; lse_q [B,K] f64 (the
  * normaliser is kept in fp64 because verification forms max(0, p - q), which a
  * common fp32 rounding of the normaliser would shift); z [B,K,V] f32.
- * Sums over the vocabulary are taken in fp64 of fp32 exponentials.
+ * The weights exp(z) that place the draw and their sums over the vocabulary
+ * are taken in fp64.
  */
 dspark_status dspark_markov_draft(const float* base_logits, const void* A, const void* Bf,
                                   dspark_dtype factor_dtype, int r, const int32_t* anchor,
@@ -154,6 +155,44 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
                             const float* u_resample, int B, int K, int V, int32_t* accepted,
                             int32_t* out_tokens, int32_t* n_out, void* workspace, size_t ws_bytes,
                             dspark_stream_t stream);
+
+/*
+ * Variant B of the round: the draft stores no z (B*K*V*4 bytes, the largest
+ * write of the round) and verification recomputes the one row of z it needs.
+ * [QbitAI] section "speculative decoding" (the residual at the first
+ * divergence needs q of that position only) and section "variable-length
+ * drafts and hardware-aware scheduling" (the whole round stays on the GPU).
+ *
+ * dspark_markov_draft_b, dspark_rnn_draft_b: the draws and the outputs
+ * draft_tokens, q_tok and lse_q of dspark_markov_draft / dspark_rnn_draft
+ * (same definition and arguments); instead of z they write op_rows [B,K,r]
+ * (bf16 bits): the operand row position i used, A[t_{b,i-1},:] for the
+ * Markov head or bf16(h_i) for the RNN head, so that
+ *   z[b,i,:] = base_logits[b,i,:] + op_rows[b,i,:] . Bf.
+ * dspark_verify_b: dspark_verify with z replaced by (base_logits, op_rows,
+ * Bf, r): the rejected row's z is recomputed on the tensor cores. Same
+ * outputs and conventions.
+ * All three need bf16 factors, r a multiple of 64 up to 256, V % 32 == 0 and
+ * B <= 512 (the tensor-core kernels); other shapes return
+ * DSPARK_ERR_UNSUPPORTED. The workspace is the one dspark_workspace_bytes sizes;
+ * dspark_verify_b uses the draft's part of it, so a draft and a verify_b on the
+ * same workspace must be ordered (one stream).
+ */
+dspark_status dspark_markov_draft_b(const float* base_logits, const void* A, const void* Bf,
+                                    dspark_dtype factor_dtype, int r, const int32_t* anchor,
+                                    const float* u_draft, int B, int K, int V, int32_t* draft_tokens,
+                                    float* q_tok, double* lse_q, uint16_t* op_rows, void* workspace,
+                                    size_t ws_bytes, dspark_stream_t stream);
+dspark_status dspark_rnn_draft_b(const float* base_logits, const void* A, const void* W, const void* Bf,
+                                 dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft,
+                                 int B, int K, int V, int32_t* draft_tokens, float* q_tok, double* lse_q,
+                                 uint16_t* op_rows, void* workspace, size_t ws_bytes, dspark_stream_t stream);
+dspark_status dspark_verify_b(const float* target_logits, const int64_t* row_start, const float* base_logits,
+                              const uint16_t* op_rows, const void* Bf, int r, const double* lse_q,
+                              const float* q_tok, const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* u_accept, const float* u_resample, int B, int K, int V,
+                              int32_t* accepted, int32_t* out_tokens, int32_t* n_out, void* workspace,
+                              size_t ws_bytes, dspark_stream_t stream);
 
 /*
  * Online calibration of the sequential temperatures from one round's outcome.
@@ -237,13 +276,17 @@ dspark_status dspark_set_wait_budget(void* workspace, uint32_t microseconds, dsp
  *                                   position 1;
  *   DSPARK_INJECT_VERIFY_BARRIER    verify skips its arrival at the first
  *                                   device-wide barrier;
+ *   DSPARK_INJECT_RESIDUAL_SLICE_SUMS  dspark_verify_b's residual kernel
+ *                                   skips its slice-sum publish of the first
+ *                                   group of requests;
  *   DSPARK_INJECT_NONE              clears the hook.
  * Pair it with a short dspark_set_wait_budget. Kept in the workspace (word 3)
  * until cleared; written on `stream`. */
 typedef enum {
   DSPARK_INJECT_NONE = 0,
   DSPARK_INJECT_DRAFT_SLICE_SUMS = 1,
-  DSPARK_INJECT_VERIFY_BARRIER = 2
+  DSPARK_INJECT_VERIFY_BARRIER = 2,
+  DSPARK_INJECT_RESIDUAL_SLICE_SUMS = 3
 } dspark_inject;
 dspark_status dspark_inject_stall(void* workspace, dspark_inject where, uint32_t cta, dspark_stream_t stream);
 

@@ -49,6 +49,12 @@ def _load() -> ctypes.CDLL:
     lib.dspark_schedule.restype = I
     lib.dspark_verify.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, P, P, P, P, Z, S]
     lib.dspark_verify.restype = I
+    lib.dspark_markov_draft_b.argtypes = [P, P, P, I, I, P, P, I, I, I, P, P, P, P, P, Z, S]
+    lib.dspark_markov_draft_b.restype = I
+    lib.dspark_rnn_draft_b.argtypes = [P, P, P, P, I, I, P, P, I, I, I, P, P, P, P, P, Z, S]
+    lib.dspark_rnn_draft_b.restype = I
+    lib.dspark_verify_b.argtypes = [P, P, P, P, P, I, P, P, P, P, P, P, I, I, I, P, P, P, P, Z, S]
+    lib.dspark_verify_b.restype = I
     lib.dspark_read_device_error.argtypes = [P, S, ctypes.POINTER(ctypes.c_uint32)]
     lib.dspark_read_device_error.restype = I
     lib.dspark_schedule_static.argtypes = [P, P, P, I, I, I, P, P, P, P, S]
@@ -147,6 +153,40 @@ def dspark_rnn_draft(base_logits, A, W, Bf, anchor, u_draft, draft_tokens, q_tok
     _check("dspark_rnn_draft", st)
 
 
+def dspark_markov_draft_b(base_logits, A, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, op_rows, workspace,
+                          stream=None) -> None:
+    """Variant B of dspark_markov_draft: no z; op_rows [B,K,r] (bfloat16)
+    receives the operand row of every position. bf16 factors only."""
+    B, K, V = base_logits.shape
+    r = A.shape[1]
+    if not (A.dtype == Bf.dtype == torch.bfloat16):
+        raise TypeError("variant B takes bf16 A and Bf")
+    st = lib.dspark_markov_draft_b(
+        _ptr(base_logits, "base_logits", torch.float32), _ptr(A, "A", numel=V * r), _ptr(Bf, "Bf", numel=r * V),
+        DSPARK_BF16, r, _ptr(anchor, "anchor", torch.int32, B), _ptr(u_draft, "u_draft", torch.float32, B * K),
+        B, K, V, _ptr(draft_tokens, "draft_tokens", torch.int32, B * K), _ptr(q_tok, "q_tok", torch.float32, B * K),
+        _ptr(lse_q, "lse_q", torch.float64, B * K), _ptr(op_rows, "op_rows", torch.bfloat16, B * K * r),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("dspark_markov_draft_b", st)
+
+
+def dspark_rnn_draft_b(base_logits, A, W, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, op_rows, workspace,
+                       stream=None) -> None:
+    """Variant B of dspark_rnn_draft (op_rows in place of z)."""
+    B, K, V = base_logits.shape
+    r = A.shape[1]
+    if not (A.dtype == Bf.dtype == W.dtype == torch.bfloat16):
+        raise TypeError("the RNN head takes bf16 A, W and Bf")
+    st = lib.dspark_rnn_draft_b(
+        _ptr(base_logits, "base_logits", torch.float32), _ptr(A, "A", numel=V * r), _ptr(W, "W", numel=r * r),
+        _ptr(Bf, "Bf", numel=r * V), DSPARK_BF16, r, _ptr(anchor, "anchor", torch.int32, B),
+        _ptr(u_draft, "u_draft", torch.float32, B * K), B, K, V,
+        _ptr(draft_tokens, "draft_tokens", torch.int32, B * K), _ptr(q_tok, "q_tok", torch.float32, B * K),
+        _ptr(lse_q, "lse_q", torch.float64, B * K), _ptr(op_rows, "op_rows", torch.bfloat16, B * K * r),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("dspark_rnn_draft_b", st)
+
+
 def dspark_schedule(conf_logits, temps, profile_ms, verify_len, survival, row_start, n_tokens, workspace,
                     stream=None) -> None:
     B, K = conf_logits.shape
@@ -191,6 +231,27 @@ def dspark_verify(target_logits, row_start, z, lse_q, q_tok, draft_tokens, verif
     _check("dspark_verify", st)
 
 
+def dspark_verify_b(target_logits, row_start, base_logits, op_rows, Bf, lse_q, q_tok, draft_tokens, verify_len,
+                    u_accept, u_resample, accepted, out_tokens, n_out, workspace, stream=None) -> None:
+    """Variant B of dspark_verify: the rejected row's z is recomputed from
+    base_logits, op_rows [B,K,r] (bfloat16) and Bf [r,V] (bfloat16)."""
+    B, K, V = base_logits.shape
+    r = Bf.shape[0]
+    if target_logits.shape[-1] != V:
+        raise ValueError("target_logits must have V columns")
+    st = lib.dspark_verify_b(
+        _ptr(target_logits, "target_logits", torch.float32), _ptr(row_start, "row_start", torch.int64, B),
+        _ptr(base_logits, "base_logits", torch.float32), _ptr(op_rows, "op_rows", torch.bfloat16, B * K * r),
+        _ptr(Bf, "Bf", torch.bfloat16, r * V), r, _ptr(lse_q, "lse_q", torch.float64, B * K),
+        _ptr(q_tok, "q_tok", torch.float32, B * K), _ptr(draft_tokens, "draft_tokens", torch.int32, B * K),
+        _ptr(verify_len, "verify_len", torch.int32, B), _ptr(u_accept, "u_accept", torch.float32, B * K),
+        _ptr(u_resample, "u_resample", torch.float32, B), B, K, V,
+        _ptr(accepted, "accepted", torch.int32, B), _ptr(out_tokens, "out_tokens", torch.int32, B * (K + 1)),
+        _ptr(n_out, "n_out", torch.int32, B), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+        _stream(stream))
+    _check("dspark_verify_b", st)
+
+
 def dspark_calibrate(conf_logits, verify_len, accepted, temps, workspace, eta: float, t_min: float, t_max: float,
                      stream=None) -> None:
     """One online step of the sequential temperatures (temps updated in place)."""
@@ -214,6 +275,7 @@ def dspark_advance_anchor(out_tokens, n_out, anchor, workspace, stream=None) -> 
 
 
 DSPARK_INJECT_NONE, DSPARK_INJECT_DRAFT_SLICE_SUMS, DSPARK_INJECT_VERIFY_BARRIER = 0, 1, 2
+DSPARK_INJECT_RESIDUAL_SLICE_SUMS = 3
 
 
 def dspark_set_wait_budget(workspace, microseconds: int, stream=None) -> None:

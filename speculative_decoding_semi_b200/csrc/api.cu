@@ -13,6 +13,7 @@ int draft_grid_size(int V, int sms);
 bool draft_tc_supported(const DraftArgs& a);
 int draft_tc_grid(int V, int sms);
 cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cudaStream_t stream);
+size_t image_bytes(int B, int r);
 }  // namespace dspark
 
 using namespace dspark;
@@ -30,6 +31,27 @@ size_t schedule_region(int B, int K) { return align_up(schedule_scratch_bytes(B,
 size_t verify_region(int B, int K, int V) { return align_up(verify_scratch_bytes(B, K, V), 256); }
 size_t scratch_bytes(int B, int K, int V, int r) {
   return schedule_region(B, K) + verify_region(B, K, V) + align_up(draft_scratch_bytes(B, K, V, r), 256);
+}
+
+// The draft's part of the scratch: part_m [B][gmax] f32, part_S [B][gmax] f64,
+// then the tensor-core kernel's extra (operand image, unit sums, RNN state).
+struct DraftScratch {
+  float* part_m;
+  double* part_S;
+  char* extra;
+};
+DraftScratch draft_scratch(char* ws, int B, int K, int V) {
+  char* scratch = ws + kScratchOffset + schedule_region(B, K) + verify_region(B, K, V);
+  const size_t gmax = std::min<size_t>(kMaxGrid, V / 8);
+  const size_t m_bytes = align_up(static_cast<size_t>(B) * gmax * sizeof(float), 256);
+  const size_t s_bytes = align_up(static_cast<size_t>(B) * gmax * sizeof(double), 256);
+  return DraftScratch{reinterpret_cast<float*>(scratch), reinterpret_cast<double*>(scratch + m_bytes),
+                      scratch + m_bytes + s_bytes};
+}
+
+// Shapes of the tensor-core kernels (variant B and the RNN head).
+bool tc_shape(dspark_dtype factor_dtype, int r, int B, int V) {
+  return factor_dtype == DSPARK_BF16 && r % 64 == 0 && r <= 256 && V % 32 == 0 && B <= 512;
 }
 
 dspark_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
@@ -52,14 +74,62 @@ dspark_status dspark_workspace_init(void* workspace, size_t ws_bytes, dspark_str
 
 namespace {
 
-// The Markov head (W == nullptr) or the RNN head (W = its recurrent weight).
+// Variant A (z) or variant B (z == nullptr: base_logits, op_rows, Bf, r).
+dspark_status verify_call(const float* target_logits, const int64_t* row_start, const float* z,
+                          const float* base_logits, const uint16_t* op_rows, const void* Bf, int r,
+                          const double* lse_q, const float* q_tok, const int32_t* draft_tokens,
+                          const int32_t* verify_len, const float* u_accept, const float* u_resample, int B, int K,
+                          int V, int32_t* accepted, int32_t* out_tokens, int32_t* n_out, void* workspace,
+                          size_t ws_bytes, dspark_stream_t stream) {
+  if (!sizes_ok(B, K, V)) return DSPARK_ERR_INVALID_ARG;
+  const void* ptrs[] = {target_logits, row_start, lse_q, q_tok, draft_tokens, verify_len,
+                        u_accept, u_resample, accepted, out_tokens, n_out, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
+  if (z != nullptr && !aligned16(z)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < kScratchOffset + schedule_region(B, K) + verify_region(B, K, V)) return DSPARK_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  VerifyArgs a{};
+  a.target = target_logits;
+  a.row_start = row_start;
+  a.z = z;
+  a.base = base_logits;
+  a.op_rows = op_rows;
+  a.Bf = Bf;
+  a.r = r;
+  if (z == nullptr) {
+    // the residual kernel's sums reuse the draft's scratch (slice sums, unit sums)
+    const DraftScratch ds = draft_scratch(ws, B, K, V);
+    a.res_part = ds.part_S;
+    a.res_unit = reinterpret_cast<double*>(ds.extra + image_bytes(B, r));
+    a.res_image = reinterpret_cast<uint8_t*>(ds.extra);
+  }
+  a.lse_q = lse_q;
+  a.q_tok = q_tok;
+  a.tokens = draft_tokens;
+  a.verify_len = verify_len;
+  a.u_accept = u_accept;
+  a.u_resample = u_resample;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.accepted = accepted;
+  a.out_tokens = out_tokens;
+  a.n_out = n_out;
+  a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
+  return from_cuda(launch_verify(a, ws + kScratchOffset + schedule_region(B, K), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// The Markov head (W == nullptr) or the RNN head (W = its recurrent weight);
+// variant A writes z, variant B (z == nullptr) writes op_rows instead.
 dspark_status draft_call(const float* base_logits, const void* A, const void* W, const void* Bf,
                          dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft, int B, int K,
-                         int V, int32_t* draft_tokens, float* q_tok, double* lse_q, float* z, void* workspace,
-                         size_t ws_bytes, dspark_stream_t stream) {
+                         int V, int32_t* draft_tokens, float* q_tok, double* lse_q, float* z, uint16_t* op_rows,
+                         void* workspace, size_t ws_bytes, dspark_stream_t stream) {
   if (!sizes_ok(B, K, V) || r < 1 || r > kMaxR) return DSPARK_ERR_INVALID_ARG;
   if (factor_dtype != DSPARK_F32 && factor_dtype != DSPARK_BF16) return DSPARK_ERR_INVALID_ARG;
-  const void* ptrs[] = {base_logits, A, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, z, workspace};
+  const void* out = z != nullptr ? static_cast<const void*>(z) : static_cast<const void*>(op_rows);
+  const void* ptrs[] = {base_logits, A, Bf, anchor, u_draft, draft_tokens, q_tok, lse_q, out, workspace};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
   if (W != nullptr && !aligned16(W)) return DSPARK_ERR_INVALID_ARG;
@@ -87,20 +157,19 @@ dspark_status draft_call(const float* base_logits, const void* A, const void* W,
   a.q_tok = q_tok;
   a.lse_q = lse_q;
   a.z = z;
+  a.op_rows = z == nullptr ? op_rows : nullptr;
   a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
   a.sync = reinterpret_cast<unsigned*>(ws + kSyncOffset);
   // bf16 factors with r % 64 == 0 (r <= 256) and V % 32 == 0 take the
   // tensor-core kernel; other shapes and fp32 factors the CUDA-core kernel
   // (which has the Markov head only)
   const bool tc = draft_tc_supported(a);
-  if (W != nullptr && !tc) return DSPARK_ERR_UNSUPPORTED;
+  if ((W != nullptr || z == nullptr) && !tc) return DSPARK_ERR_UNSUPPORTED;
   const int G = tc ? draft_tc_grid(V, sms) : draft_grid_size(V, sms);
-  char* scratch = ws + kScratchOffset + schedule_region(B, K) + verify_region(B, K, V);
-  const size_t gmax = std::min<size_t>(kMaxGrid, V / 8);
-  a.part_m = reinterpret_cast<float*>(scratch);
-  a.part_S = reinterpret_cast<double*>(scratch + align_up(static_cast<size_t>(B) * gmax * sizeof(float), 256));
-  char* extra = scratch + align_up(static_cast<size_t>(B) * gmax * sizeof(float), 256) +
-                align_up(static_cast<size_t>(B) * gmax * sizeof(double), 256);
+  const DraftScratch ds = draft_scratch(ws, B, K, V);
+  a.part_m = ds.part_m;
+  a.part_S = ds.part_S;
+  char* extra = ds.extra;
 
   cudaError_t e = cudaMemsetAsync(a.sync, 0, kSyncBytes, s);
   if (e != cudaSuccess) return DSPARK_ERR_CUDA;
@@ -116,17 +185,39 @@ dspark_status dspark_markov_draft(const float* base_logits, const void* A, const
                                   const float* u_draft, int B, int K, int V, int32_t* draft_tokens,
                                   float* q_tok, double* lse_q, float* z, void* workspace,
                                   size_t ws_bytes, dspark_stream_t stream) {
+  if (z == nullptr) return DSPARK_ERR_INVALID_ARG;
   return draft_call(base_logits, A, nullptr, Bf, factor_dtype, r, anchor, u_draft, B, K, V, draft_tokens, q_tok,
-                    lse_q, z, workspace, ws_bytes, stream);
+                    lse_q, z, nullptr, workspace, ws_bytes, stream);
 }
 
 dspark_status dspark_rnn_draft(const float* base_logits, const void* A, const void* W, const void* Bf,
                                dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft, int B,
                                int K, int V, int32_t* draft_tokens, float* q_tok, double* lse_q, float* z,
                                void* workspace, size_t ws_bytes, dspark_stream_t stream) {
-  if (W == nullptr) return DSPARK_ERR_INVALID_ARG;
+  if (W == nullptr || z == nullptr) return DSPARK_ERR_INVALID_ARG;
   return draft_call(base_logits, A, W, Bf, factor_dtype, r, anchor, u_draft, B, K, V, draft_tokens, q_tok, lse_q, z,
-                    workspace, ws_bytes, stream);
+                    nullptr, workspace, ws_bytes, stream);
+}
+
+dspark_status dspark_markov_draft_b(const float* base_logits, const void* A, const void* Bf,
+                                    dspark_dtype factor_dtype, int r, const int32_t* anchor,
+                                    const float* u_draft, int B, int K, int V, int32_t* draft_tokens,
+                                    float* q_tok, double* lse_q, uint16_t* op_rows, void* workspace,
+                                    size_t ws_bytes, dspark_stream_t stream) {
+  if (op_rows == nullptr) return DSPARK_ERR_INVALID_ARG;
+  if (sizes_ok(B, K, V) && r >= 1 && !tc_shape(factor_dtype, r, B, V)) return DSPARK_ERR_UNSUPPORTED;
+  return draft_call(base_logits, A, nullptr, Bf, factor_dtype, r, anchor, u_draft, B, K, V, draft_tokens, q_tok,
+                    lse_q, nullptr, op_rows, workspace, ws_bytes, stream);
+}
+
+dspark_status dspark_rnn_draft_b(const float* base_logits, const void* A, const void* W, const void* Bf,
+                                 dspark_dtype factor_dtype, int r, const int32_t* anchor, const float* u_draft,
+                                 int B, int K, int V, int32_t* draft_tokens, float* q_tok, double* lse_q,
+                                 uint16_t* op_rows, void* workspace, size_t ws_bytes, dspark_stream_t stream) {
+  if (W == nullptr || op_rows == nullptr) return DSPARK_ERR_INVALID_ARG;
+  if (sizes_ok(B, K, V) && r >= 1 && !tc_shape(factor_dtype, r, B, V)) return DSPARK_ERR_UNSUPPORTED;
+  return draft_call(base_logits, A, W, Bf, factor_dtype, r, anchor, u_draft, B, K, V, draft_tokens, q_tok, lse_q,
+                    nullptr, op_rows, workspace, ws_bytes, stream);
 }
 
 dspark_status dspark_schedule(const float* conf_logits, const float* temps, const float* profile_ms,
@@ -161,31 +252,26 @@ dspark_status dspark_verify(const float* target_logits, const int64_t* row_start
                             const int32_t* verify_len, const float* u_accept, const float* u_resample,
                             int B, int K, int V, int32_t* accepted, int32_t* out_tokens, int32_t* n_out,
                             void* workspace, size_t ws_bytes, dspark_stream_t stream) {
-  if (!sizes_ok(B, K, V)) return DSPARK_ERR_INVALID_ARG;
-  const void* ptrs[] = {target_logits, row_start, z, lse_q, q_tok, draft_tokens, verify_len,
-                        u_accept, u_resample, accepted, out_tokens, n_out, workspace};
-  for (const void* p : ptrs)
-    if (p == nullptr || !aligned16(p)) return DSPARK_ERR_INVALID_ARG;
-  if (ws_bytes < kScratchOffset + schedule_region(B, K) + verify_region(B, K, V)) return DSPARK_ERR_INVALID_ARG;
-  char* ws = static_cast<char*>(workspace);
-  VerifyArgs a{};
-  a.target = target_logits;
-  a.row_start = row_start;
-  a.z = z;
-  a.lse_q = lse_q;
-  a.q_tok = q_tok;
-  a.tokens = draft_tokens;
-  a.verify_len = verify_len;
-  a.u_accept = u_accept;
-  a.u_resample = u_resample;
-  a.B = B;
-  a.K = K;
-  a.V = V;
-  a.accepted = accepted;
-  a.out_tokens = out_tokens;
-  a.n_out = n_out;
-  a.err = reinterpret_cast<unsigned*>(ws + kErrOffset);
-  return from_cuda(launch_verify(a, ws + kScratchOffset + schedule_region(B, K), reinterpret_cast<cudaStream_t>(stream)));
+  if (z == nullptr) return DSPARK_ERR_INVALID_ARG;
+  return verify_call(target_logits, row_start, z, nullptr, nullptr, nullptr, 0, lse_q, q_tok, draft_tokens,
+                     verify_len, u_accept, u_resample, B, K, V, accepted, out_tokens, n_out, workspace, ws_bytes,
+                     stream);
+}
+
+dspark_status dspark_verify_b(const float* target_logits, const int64_t* row_start, const float* base_logits,
+                              const uint16_t* op_rows, const void* Bf, int r, const double* lse_q,
+                              const float* q_tok, const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* u_accept, const float* u_resample, int B, int K, int V,
+                              int32_t* accepted, int32_t* out_tokens, int32_t* n_out, void* workspace,
+                              size_t ws_bytes, dspark_stream_t stream) {
+  if (base_logits == nullptr || op_rows == nullptr || Bf == nullptr) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(base_logits) || !aligned16(op_rows) || !aligned16(Bf)) return DSPARK_ERR_INVALID_ARG;
+  if (r < 1 || r > kMaxR) return DSPARK_ERR_INVALID_ARG;
+  if (sizes_ok(B, K, V) && !tc_shape(DSPARK_BF16, r, B, V)) return DSPARK_ERR_UNSUPPORTED;
+  if (ws_bytes < dspark_workspace_bytes(B, K, V, r)) return DSPARK_ERR_INVALID_ARG;
+  return verify_call(target_logits, row_start, nullptr, base_logits, op_rows, Bf, r, lse_q, q_tok, draft_tokens,
+                     verify_len, u_accept, u_resample, B, K, V, accepted, out_tokens, n_out, workspace, ws_bytes,
+                     stream);
 }
 
 dspark_status dspark_set_wait_budget(void* workspace, uint32_t microseconds, dspark_stream_t stream) {
@@ -197,7 +283,8 @@ dspark_status dspark_set_wait_budget(void* workspace, uint32_t microseconds, dsp
 
 dspark_status dspark_inject_stall(void* workspace, dspark_inject where, uint32_t cta, dspark_stream_t stream) {
   if (workspace == nullptr || !aligned16(workspace)) return DSPARK_ERR_INVALID_ARG;
-  if (where != DSPARK_INJECT_NONE && where != DSPARK_INJECT_DRAFT_SLICE_SUMS && where != DSPARK_INJECT_VERIFY_BARRIER)
+  if (where != DSPARK_INJECT_NONE && where != DSPARK_INJECT_DRAFT_SLICE_SUMS && where != DSPARK_INJECT_VERIFY_BARRIER &&
+      where != DSPARK_INJECT_RESIDUAL_SLICE_SUMS)
     return DSPARK_ERR_INVALID_ARG;
   if (cta >= (1u << 24)) return DSPARK_ERR_INVALID_ARG;
   const uint32_t v = where == DSPARK_INJECT_NONE ? 0u : ((static_cast<uint32_t>(where) << 24) | cta);

@@ -170,4 +170,187 @@ __device__ __noinline__ void select_token(const DraftArgs& a, int b, int i, int 
   Sync::sync();
 }
 
+// Among n values x(0..n-1) (read through `get`) laid out in lane-contiguous
+// blocks, find the first index whose inclusive prefix exceeds `thr(total)`
+// (strict, never a zero entry); returns it, or the last positive index if
+// rounding leaves none, with its exclusive prefix in *excl and the sum of all
+// n values in *total. `thr` maps the total to the threshold, so one pass both
+// sums and searches. Sums run sequentially within a lane's block and in lane
+// order across blocks. One warp, all lanes; each lane's loads are issued
+// together (up to kSearchRegs values per lane stay in registers).
+template <int kSearchRegs, class Get, class Thr>
+__device__ __forceinline__ int warp_search(int n, Get get, Thr thr_of, int lane, double* excl, double* total) {
+  const int per = (n + 31) / 32;
+  const int lo = min(n, lane * per), hi = min(n, lo + per);
+  double local = 0.0;
+  int last_pos = -1;
+  double vals[kSearchRegs];
+  const bool in_regs = per <= kSearchRegs;
+  if (in_regs) {
+#pragma unroll
+    for (int j = 0; j < kSearchRegs; ++j) vals[j] = get(min(lo + j, n - 1));  // clamped: the loads issue together
+#pragma unroll
+    for (int j = 0; j < kSearchRegs; ++j)
+      if (lo + j >= hi) vals[j] = 0.0;
+#pragma unroll
+    for (int j = 0; j < kSearchRegs; ++j) {
+      local += vals[j];
+      if (vals[j] > 0.0) last_pos = lo + j;
+    }
+  } else {
+    for (int x = lo; x < hi; ++x) {
+      const double v = get(x);
+      local += v;
+      if (v > 0.0) last_pos = x;
+    }
+  }
+  double inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double nb = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += nb;
+  }
+  double mine = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) mine = 0.0;
+  *total = __shfl_sync(0xffffffffu, inc, 31);
+  const double thr = thr_of(*total);
+  int found = 0x7fffffff;
+  double found_ex = 0.0;
+  if (lo < hi && mine + local > thr) {
+    double c = mine;
+    if (in_regs) {
+#pragma unroll
+      for (int j = 0; j < kSearchRegs; ++j) {
+        if (found == 0x7fffffff && lo + j < hi) {
+          if (c + vals[j] > thr && vals[j] > 0.0) {
+            found = lo + j;
+            found_ex = c;
+          }
+          c += vals[j];
+        }
+      }
+    } else {
+      for (int x = lo; x < hi; ++x) {
+        const double v = get(x);
+        if (c + v > thr && v > 0.0) {
+          found = x;
+          found_ex = c;
+          break;
+        }
+        c += v;
+      }
+    }
+  }
+  int best = found;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if (best == 0x7fffffff) {
+    // rounding: the last positive entry, with its exclusive prefix from its owner
+    int lp = last_pos;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lp = max(lp, __shfl_xor_sync(0xffffffffu, lp, o));
+    best = max(lp, 0);
+    double e = 0.0;
+    if (best >= lo && best < hi) {
+      e = mine;
+      for (int x = lo; x < best; ++x) e += get(x);
+    }
+    const int owner = per > 0 ? min(31, best / per) : 0;
+    *excl = __shfl_sync(0xffffffffu, e, owner);
+    return best;
+  }
+  const int owner = per > 0 ? min(31, best / per) : 0;
+  *excl = __shfl_sync(0xffffffffu, found_ex, owner);
+  return best;
+}
+
+
+// Sum over the 32 lanes of a warp of 32 values per lane, v[c] for c = 0..31,
+// by a halving exchange: lane l returns the total of v[l] (31 exchanges).
+__device__ __forceinline__ float warp_transpose_sum32f(float (&v)[32], int lane) {
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int half = 16 >> step, bit = 16 >> step;
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+    }
+  }
+  return v[0];
+}
+
+// z of row v0 + lane of one row of logits, base + a . Bf, for a 32-row unit
+// at v0 (a multiple of 32): a is the operand row (r bf16 values), Bf the
+// [r, V] factor (bf16), zbase the row's base logits. fp32 (one warp; lane l
+// takes the rank indices l, l + 32, ... and the lanes' 32 partial sums are
+// exchanged at the end). For r a multiple of 32.
+static __device__ __noinline__ float unit_logit(const uint16_t* a, const uint16_t* Bf, const float* zbase, int r, int V,
+                                                long long v0, int lane) {
+  float acc[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+#pragma unroll 2
+  for (int k = lane; k < r; k += 32) {
+    const float ak = __uint_as_float(static_cast<unsigned>(__ldcg(a + k)) << 16);
+    const uint4* row = reinterpret_cast<const uint4*>(Bf + static_cast<long long>(k) * V + v0);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = __ldg(row + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[8 * c + 2 * j] = fmaf(ak, __uint_as_float(w[j] << 16), acc[8 * c + 2 * j]);
+        acc[8 * c + 2 * j + 1] = fmaf(ak, __uint_as_float(w[j] & 0xffff0000u), acc[8 * c + 2 * j + 1]);
+      }
+    }
+  }
+  const float bias = warp_transpose_sum32f(acc, lane);
+  return __fadd_rn(__ldcg(zbase + v0 + lane), bias);
+}
+
+// Stage the 32 columns v0.. of the [r, V] bf16 factor Bf in shared memory as
+// [r][32] (64 bytes a row), one warp: 16-byte cp.async copies, r * 4 of them,
+// all issued at once so the unit arrives in one memory trip; then
+// stage_unit_wait. v0 is a multiple of 32, V of 32; dst 16-byte aligned.
+__device__ __forceinline__ void stage_unit_issue(uint8_t* dst, const uint16_t* Bf, int V, int r, long long v0,
+                                                 int lane) {
+  for (int idx = lane; idx < r * 4; idx += 32) {
+    const int k = idx >> 2, c = idx & 3;
+    const uint16_t* src = Bf + static_cast<long long>(k) * V + v0 + 8 * c;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(
+                     dst + k * 64 + c * 16))),
+                 "l"(src)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void stage_unit_wait() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();  // every lane's copies are visible to the warp
+}
+
+// sum_k a_k Bf[k, v0 + lane] over a 32-column unit staged in shared memory:
+// bfu [r][32] bf16 (stage_unit_issue), a_s the operand row (r bf16, 16-byte
+// aligned). fp32, eight partial sums (k mod 8) added at the end.
+__device__ __forceinline__ float staged_unit_dot(const uint16_t* bfu, const uint4* a_s, int r, int lane) {
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int k0 = 0; k0 < r; k0 += 8) {
+    const uint4 av = a_s[k0 >> 3];
+    const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float b0 = __uint_as_float(static_cast<unsigned>(bfu[(k0 + 2 * j) * 32 + lane]) << 16);
+      const float b1 = __uint_as_float(static_cast<unsigned>(bfu[(k0 + 2 * j + 1) * 32 + lane]) << 16);
+      acc[2 * j] = fmaf(__uint_as_float(aw[j] << 16), b0, acc[2 * j]);
+      acc[2 * j + 1] = fmaf(__uint_as_float(aw[j] & 0xffff0000u), b1, acc[2 * j + 1]);
+    }
+  }
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
 }  // namespace dspark

@@ -10,20 +10,19 @@
 //
 // One persistent cooperative kernel, one CTA per SM; CTA g owns the vocabulary
 // slice chunk_bounds(V, 32, G, g) for every request. Requests are split into
-// groups (of up to 128) that synchronise independently, so while one group's
-// tokens are being drawn the CTA streams another group's logits. Warp roles:
-//   warps 0-7  epilogue: read the accumulator (warp w reads TMEM lanes
-//              32*(w%4).. = vocabulary rows; columns = requests), add the base
-//              logits staged by TMA, write z back through TMA, and sum exp(z)
-//              in fp64 per request over each 32-row unit (reading the staged
-//              box across its rows) and over the CTA's slice;
-//   warp 8     TMA producer of Bf tiles (ring of stages, L2 evict-last so the
+// groups (of up to 128) that synchronise independently. Warp roles:
+//   warps 0-15 epilogue, four per TMEM lane quadrant: read the accumulator
+//              (warp w reads TMEM lanes 32*(w%4).. = vocabulary rows; columns
+//              = requests, 16 at a time), add the base logits staged by TMA,
+//              write z back through TMA, and sum exp(z) in fp64 per request
+//              over each 32-row unit and over the CTA's slice;
+//   warp 16    TMA producer of Bf tiles (ring of stages, L2 evict-last so the
 //              78 MB factor can stay resident across positions);
-//   warp 9     TMEM owner and MMA issuer (M = 128 vocabulary rows, N = the
+//   warp 17    TMEM owner and MMA issuer (M = 128 vocabulary rows, N = the
 //              group's requests, K = r in steps of 16); it bulk-loads each
 //              group's operand (the A rows of the last drawn tokens, already
 //              in MMA layout) once the group's tokens are published;
-//   warp 10    selector: publishes the slice sums, waits for every CTA, draws
+//   warp 18    selector: publishes the slice sums, waits for every CTA, draws
 //              the tokens of its requests (b mod G == g) by a three-level
 //              inverse-CDF search (the G slice sums, the chosen slice's unit
 //              sums, then the chosen unit's 32 weights), writes the A rows of
@@ -31,6 +30,10 @@
 //              group's tokens before releasing the next position.
 // The epilogue streams base and z through per-warp TMA rings (L2 evict-first)
 // that run ahead across positions, since they do not depend on the tokens.
+// Variant B writes no z (the ring carries base only): the selector keeps the
+// operand row of every position in op_rows instead, and the last search level
+// recomputes its unit's 32 logits from base, that row and Bf. The verify of
+// variant B recomputes the one rejected row of z the same way.
 // Weights. z = base + bias is rounded to fp32 for the output, but the weight
 // is exp(base + bias) in fp64 (exp_sum2: the reduced argument is built from
 // base and bias, so z's rounding never enters; relative error ~5e-9) with a
@@ -97,18 +100,23 @@ struct TcParams {
   double* unit_sum;     // [V/32][B] sums of exp(z) over each 32-row unit, this position
   double* hstate;       // [B][r] RNN head: state h_i of each request (fp64)
   double* ustate;       // [B][r] RNN head: W h_i, formed while position i streams
+  uint16_t* op_rows;    // [B][K][r] variant B: the operand row of every position (bf16), or null
+  int sel_bytes;        // variant B: shared staging of the last search level (0 in variant A)
 };
 
 struct Layout {
-  int bf, brows, ring, part, bar, tab, misc, total;
+  int bf, brows, ring, sel, part, bar, tab, misc, total;
 };
 
-__host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs, int part_bytes) {
+// sel_bytes: variant B's staging of one unit's Bf columns and operand row for
+// the last search level (0 in variant A)
+__host__ __device__ inline Layout make_layout(int nbf, int brows_bytes, int nbs, int part_bytes, int sel_bytes) {
   Layout L;
   L.bf = 0;
   L.brows = L.bf + nbf * kBfStageBytes;
   L.ring = L.brows + ((brows_bytes + 1023) / 1024) * 1024;
-  L.part = L.ring + kEpiWarps * nbs * kBoxBytes;
+  L.sel = L.ring + kEpiWarps * nbs * kBoxBytes;
+  L.part = L.sel + ((sel_bytes + 127) / 128) * 128;
   L.bar = L.part + ((part_bytes + 15) / 16) * 16;
   L.tab = L.bar + kBarBytes;
   L.misc = L.tab + 16 * 8;
@@ -198,101 +206,6 @@ struct Items {
   }
 };
 
-// Among n values x(0..n-1) (read through `get`) laid out in lane-contiguous
-// blocks, find the first index whose inclusive prefix exceeds `thr(total)`
-// (strict, never a zero entry); returns it, or the last positive index if
-// rounding leaves none, with its exclusive prefix in *excl and the sum of all
-// n values in *total. `thr` maps the total to the threshold, so one pass both
-// sums and searches. Sums run sequentially within a lane's block and in lane
-// order across blocks. One warp, all lanes; each lane's loads are issued
-// together (up to kSearchRegs values per lane stay in registers).
-template <int kSearchRegs, class Get, class Thr>
-__device__ __forceinline__ int warp_search(int n, Get get, Thr thr_of, int lane, double* excl, double* total) {
-  const int per = (n + 31) / 32;
-  const int lo = min(n, lane * per), hi = min(n, lo + per);
-  double local = 0.0;
-  int last_pos = -1;
-  double vals[kSearchRegs];
-  const bool in_regs = per <= kSearchRegs;
-  if (in_regs) {
-#pragma unroll
-    for (int j = 0; j < kSearchRegs; ++j) vals[j] = get(min(lo + j, n - 1));  // clamped: the loads issue together
-#pragma unroll
-    for (int j = 0; j < kSearchRegs; ++j)
-      if (lo + j >= hi) vals[j] = 0.0;
-#pragma unroll
-    for (int j = 0; j < kSearchRegs; ++j) {
-      local += vals[j];
-      if (vals[j] > 0.0) last_pos = lo + j;
-    }
-  } else {
-    for (int x = lo; x < hi; ++x) {
-      const double v = get(x);
-      local += v;
-      if (v > 0.0) last_pos = x;
-    }
-  }
-  double inc = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double nb = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += nb;
-  }
-  double mine = __shfl_up_sync(0xffffffffu, inc, 1);
-  if (lane == 0) mine = 0.0;
-  *total = __shfl_sync(0xffffffffu, inc, 31);
-  const double thr = thr_of(*total);
-  int found = 0x7fffffff;
-  double found_ex = 0.0;
-  if (lo < hi && mine + local > thr) {
-    double c = mine;
-    if (in_regs) {
-#pragma unroll
-      for (int j = 0; j < kSearchRegs; ++j) {
-        if (found == 0x7fffffff && lo + j < hi) {
-          if (c + vals[j] > thr && vals[j] > 0.0) {
-            found = lo + j;
-            found_ex = c;
-          }
-          c += vals[j];
-        }
-      }
-    } else {
-      for (int x = lo; x < hi; ++x) {
-        const double v = get(x);
-        if (c + v > thr && v > 0.0) {
-          found = x;
-          found_ex = c;
-          break;
-        }
-        c += v;
-      }
-    }
-  }
-  int best = found;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
-  if (best == 0x7fffffff) {
-    // rounding: the last positive entry, with its exclusive prefix from its owner
-    int lp = last_pos;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lp = max(lp, __shfl_xor_sync(0xffffffffu, lp, o));
-    best = max(lp, 0);
-    double e = 0.0;
-    if (best >= lo && best < hi) {
-      e = mine;
-      for (int x = lo; x < best; ++x) e += get(x);
-    }
-    const int owner = per > 0 ? min(31, best / per) : 0;
-    *excl = __shfl_sync(0xffffffffu, e, owner);
-    return best;
-  }
-  const int owner = per > 0 ? min(31, best / per) : 0;
-  *excl = __shfl_sync(0xffffffffu, found_ex, owner);
-  return best;
-}
-
-
 // Draw from the whole row z with its exact maximum as the shift, for a row
 // whose sum of exp(z) leaves [1e-30, 1e30] (one warp). Non-finite logits are
 // recorded as a device error and give token 0.
@@ -317,15 +230,93 @@ __device__ __noinline__ int draw_full_row(const float* zrow, int V, double u, in
   return tok;
 }
 
+// Variant B (z not stored): z of row 32 ux + lane for request b at position
+// i, recomputed from the operand row the position used.
+__device__ __forceinline__ float unit_z(const TcParams& p, int b, int i, int ux, int lane) {
+  const DraftArgs& d = p.d;
+  const long long o = static_cast<long long>(b) * d.K + i;
+  return unit_logit(p.op_rows + o * d.r, static_cast<const uint16_t*>(d.Bf), d.base + o * d.V, d.r, d.V,
+                    static_cast<long long>(ux) * kUnit, lane);
+}
+
+// Variant B, for a row whose sum of exp(z) leaves the fixed-shift range: the
+// draw of draw_full_row over z recomputed one 32-row unit at a time (three
+// passes over the row: its maximum, its sum, the search). Slow, and only for
+// rows with logits beyond about +-640.
+__device__ __noinline__ int draw_full_row_b(const TcParams& p, int b, int i, double u, int lane, double* w_t,
+                                            float* shift, double* W) {
+  const DraftArgs& d = p.d;
+  const int nu = d.V / kUnit;
+  float mx = -INFINITY;
+  for (int ux = 0; ux < nu; ++ux) mx = fmaxf(mx, unit_z(p, b, i, ux, lane));
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+  *shift = mx;
+  double tot = 0.0;
+  for (int ux = 0; ux < nu; ++ux) tot += warp_sum(static_cast<double>(expf(unit_z(p, b, i, ux, lane) - mx)));
+  *W = tot;
+  if (!(tot > 0.0) || !(tot < INFINITY)) {
+    if (lane == 0) set_error(d.err, DSPARK_ERR_DEVICE_ASSERT, 0x30000000u | static_cast<unsigned>(b));
+    *w_t = 0.0;
+    *W = 1.0;
+    return 0;
+  }
+  const double thr = u * tot;
+  double c = 0.0;
+  int last = -1, last_ux = 0;
+  for (int ux = 0; ux < nu; ++ux) {
+    const double w = static_cast<double>(expf(unit_z(p, b, i, ux, lane) - mx));
+    const double s = warp_sum(w);
+    const unsigned pos = __ballot_sync(0xffffffffu, w > 0.0);
+    if (pos) {
+      last = 31 - __clz(pos);
+      last_ux = ux;
+    }
+    if (c + s > thr) {
+      const double inc = c + warp_inclusive_scan(w);
+      const unsigned hit = __ballot_sync(0xffffffffu, inc > thr && w > 0.0);
+      if (hit) {
+        const int x = __ffs(hit) - 1;
+        *w_t = __shfl_sync(0xffffffffu, w, x);
+        return ux * kUnit + x;
+      }
+    }
+    c += s;
+  }
+  // rounding: the last positive weight of the row
+  const float zl = unit_z(p, b, i, last_ux, lane);
+  *w_t = __shfl_sync(0xffffffffu, static_cast<double>(expf(zl - mx)), max(last, 0));
+  return last_ux * kUnit + max(last, 0);
+}
+
 // Draw request b's token at position i (one warp) by a three-level
 // inverse-CDF search over fp64 sums of the weights exp(z): the G slice sums
 // (whose total is the W that u scales), the chosen slice's sums over its 32-row
-// units, then the chosen unit's 32 weights (from the stored fp32 z). Writes
-// draft_tokens, q_tok and lse_q; returns the token.
-__device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane, const double* t16) {
+// units, then the chosen unit's 32 weights (from the stored fp32 z, or in
+// variant B from z recomputed for that unit). Writes draft_tokens, q_tok and
+// lse_q; returns the token.
+// Variant B: z of row 32 ux + lane for request b at position i, from the
+// unit's Bf columns staged in shared memory (`sel`: r x 32 bf16, then the
+// operand row) and the position's operand row: base + sum_k a_k Bf[k, v].
+__device__ __forceinline__ float unit_z_staged(const TcParams& p, int b, int i, int ux, int lane, uint8_t* sel) {
   const DraftArgs& d = p.d;
   const long long o = static_cast<long long>(b) * d.K + i;
-  const float* zrow = d.z + o * d.V;
+  const long long v0 = static_cast<long long>(ux) * kUnit;
+  stage_unit_issue(sel, static_cast<const uint16_t*>(d.Bf), d.V, d.r, v0, lane);
+  const float zb = __ldcg(d.base + o * d.V + v0 + lane);
+  uint4* a_s = reinterpret_cast<uint4*>(sel + d.r * kUnit * 2);
+  if (lane < d.r / 8) a_s[lane] = __ldcg(reinterpret_cast<const uint4*>(p.op_rows + o * d.r) + lane);
+  stage_unit_wait();
+  const float acc = staged_unit_dot(reinterpret_cast<const uint16_t*>(sel), a_s, d.r, lane);
+  __syncwarp();  // every lane has read the staging before it is reused
+  return __fadd_rn(zb, acc);
+}
+
+template <bool kStoreZ>
+__device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane, const double* t16,
+                                        uint8_t* sel) {
+  const DraftArgs& d = p.d;
+  const long long o = static_cast<long long>(b) * d.K + i;
   const double u = static_cast<double>(d.u[o]);
   const double* part = d.part_S + static_cast<long long>(b) * G;
   double ex, W;
@@ -349,7 +340,9 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
                              [&](double) { return R; }, lane, &ex2, &tot2);
     const double R2 = R - ex2;
     // level 3: the unit's weights, one per lane
-    const double w = exp_fine(__ldcg(zrow + static_cast<long long>(ux) * kUnit + lane), 0.f, t16);
+    const float zu = kStoreZ ? __ldcg(d.z + o * d.V + static_cast<long long>(ux) * kUnit + lane)
+                             : unit_z_staged(p, b, i, ux, lane, sel);
+    const double w = exp_fine(zu, 0.f, t16);
     const double inc = warp_inclusive_scan(w);
     const unsigned hit = __ballot_sync(0xffffffffu, inc > R2 && w > 0.0);
     const unsigned pos = __ballot_sync(0xffffffffu, w > 0.0);
@@ -357,8 +350,10 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
     const int x = hit ? __ffs(hit) - 1 : (pos ? 31 - __clz(pos) : 0);
     w_t = __shfl_sync(0xffffffffu, w, x);
     tok = ux * kUnit + x;
+  } else if (kStoreZ) {
+    tok = draw_full_row(d.z + o * d.V, d.V, u, lane, b, d.err, &w_t, &shift, &W);
   } else {
-    tok = draw_full_row(zrow, d.V, u, lane, b, d.err, &w_t, &shift, &W);
+    tok = draw_full_row_b(p, b, i, u, lane, &w_t, &shift, &W);
   }
   if (lane == 0) {
     d.tokens[o] = tok;
@@ -368,9 +363,10 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
   return tok;
 }
 
-// A row of the MMA's B operand for request b: A[t, :] into the operand image
-// of b's group, K-major with the 128-byte swizzle (one warp).
-__device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t, int lane) {
+// A row of the MMA's B operand for request b at position pos: A[t, :] into
+// the operand image of b's group, K-major with the 128-byte swizzle, and in
+// variant B also into op_rows (one warp).
+__device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t, int pos, int lane) {
   const int gr = b / p.gsize, n = b - gr * p.gsize;
   const int N = round16(group_real(p, gr));
   const int cpr = p.d.r / 8;
@@ -380,6 +376,8 @@ __device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t,
     const uint4 v = __ldg(A4 + ch);
     const int kb = ch >> 3, c = ch & 7;
     *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) = v;
+    if (p.op_rows != nullptr)
+      reinterpret_cast<uint4*>(p.op_rows + (static_cast<long long>(b) * p.d.K + pos) * p.d.r)[ch] = v;
   }
 }
 
@@ -449,8 +447,9 @@ __device__ __noinline__ void rnn_matvec(const TcParams& p, int b, int lane) {
 }
 
 // h = tanh(A[t] + U) (U = W h_prev, or 0 at the first position) for request
-// b: stored as the new state and written, rounded to bf16, as b's operand row.
-__device__ __noinline__ void rnn_step(const TcParams& p, int b, int t, bool first, int lane) {
+// b: stored as the new state and written, rounded to bf16, as b's operand row
+// of position pos (and in variant B into op_rows).
+__device__ __noinline__ void rnn_step(const TcParams& p, int b, int t, bool first, int pos, int lane) {
   const int r = p.d.r, nch = r / 8;
   if (lane >= nch) return;
   const int gr = b / p.gsize, n = b - gr * p.gsize;
@@ -471,8 +470,10 @@ __device__ __noinline__ void rnn_step(const TcParams& p, int b, int t, bool firs
   }
   uint8_t* img = p.image + static_cast<long long>(gr) * p.image_stride;
   const int kb = lane >> 3, c = lane & 7;
-  *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
-      make_uint4(out[0], out[1], out[2], out[3]);
+  const uint4 row = make_uint4(out[0], out[1], out[2], out[3]);
+  *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) = row;
+  if (p.op_rows != nullptr)
+    reinterpret_cast<uint4*>(p.op_rows + (static_cast<long long>(b) * p.d.K + pos) * p.d.r)[lane] = row;
 }
 
 // One warp: every lane waits for *ctr >= target (bounded), so the warp stays
@@ -486,14 +487,14 @@ __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned 
 }
 
 // 19 warps: five share a 16K-register SM sub-partition, so at most 96 registers each
-template <bool kRnn>
+template <bool kRnn, bool kStoreZ>
 __global__ void __maxnreg__(96)
     draft_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_bf,
                     const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_z) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const DraftArgs& d = p.d;
-  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, p.ngroups * 4 * p.gsize * 8);
+  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, p.ngroups * 4 * p.gsize * 8, p.sel_bytes);
   Bars bars = carve_bars(smem + Ly.bar);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
@@ -660,8 +661,8 @@ __global__ void __maxnreg__(96)
     bool ok = true;
     // position 0's operand: the anchors' rows, and zeros in padded rows
     for (int b = g; b < d.B; b += G) {
-      if (kRnn) rnn_step(p, b, previous_token(d, b, 0), true, lane);
-      else write_image_row(p, b, previous_token(d, b, 0), lane);
+      if (kRnn) rnn_step(p, b, previous_token(d, b, 0), true, 0, lane);
+      else write_image_row(p, b, previous_token(d, b, 0), 0, lane);
     }
     if (g == 0) {
       for (int gr = 0; gr < p.ngroups; ++gr) {
@@ -720,10 +721,10 @@ __global__ void __maxnreg__(96)
           ok = warp_wait_counter(&p.sync_part[slot], static_cast<unsigned>(G), d.err, 0x600u + slot, s_abort, lane);
           if (!ok) break;
           for (int b = first; b < gbase + nreal; b += G) {
-            const int t = select_warp(p, b, i, G, lane, t16);
+            const int t = select_warp<kStoreZ>(p, b, i, G, lane, t16, smem + Ly.sel);
             if (i + 1 < d.K) {
-              if (kRnn) rnn_step(p, b, t, false, lane);
-              else write_image_row(p, b, t, lane);
+              if (kRnn) rnn_step(p, b, t, false, i + 1, lane);
+              else write_image_row(p, b, t, i + 1, lane);
             }
             ++mine;
           }
@@ -838,14 +839,16 @@ __global__ void __maxnreg__(96)
                     const F2 x = f2(box[c * kUnit + lane], box[(c + 1) * kUnit + lane]);
                     const F2 y = f2(__uint_as_float(rg[c]), __uint_as_float(rg[c + 1]));
                     const F2 zh = add2(x, y);
-                    box[c * kUnit + lane] = f2_lo(zh);
-                    box[(c + 1) * kUnit + lane] = f2_hi(zh);
+                    if (kStoreZ) {
+                      box[c * kUnit + lane] = f2_lo(zh);
+                      box[(c + 1) * kUnit + lane] = f2_hi(zh);
+                    }
                     exp_sum2(x, y, zh, t16, &wv[c], &wv[c + 1]);
                   }
-                  fence_proxy_async_shared();
+                  if (kStoreZ) fence_proxy_async_shared();
                   __syncwarp();
                   ++nc;
-                  if (lane == 0) {
+                  if (kStoreZ && lane == 0) {
                     tma_store_3d(&tm_z, box, v0, i, gbase + col0, pol_first);
                     bulk_commit();
                   }
@@ -904,20 +907,6 @@ __global__ void __maxnreg__(96)
   }
 }
 
-using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<EncodeFn>(nullptr);
-    return reinterpret_cast<EncodeFn>(f);
-  }();
-  return fn;
-}
-
 // Requests per group: up to 128, a multiple of 32 so that a group's z boxes
 // never reach into the next group. Batches that fit one group are not split:
 // with two groups each group's hand-offs meet the other group's stream on
@@ -949,7 +938,7 @@ size_t draft_tc_extra_bytes(int B, int V, int r) {
 }
 
 cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cudaStream_t stream) {
-  EncodeFn enc = encode_fn();
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
   TcParams p{};
   p.d = a;
@@ -965,17 +954,19 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
   p.unit_sum = reinterpret_cast<double*>(extra + image_bytes(a.B, a.r));
   p.hstate = reinterpret_cast<double*>(extra + image_bytes(a.B, a.r) + unit_sum_bytes(a.B, a.V));
   p.ustate = p.hstate + rnn_state_bytes(a.B, a.r) / sizeof(double);
+  p.op_rows = a.op_rows;
   p.sync_part = sync;
   p.sync_tok = sync + a.K * p.ngroups;
   int dev = 0, max_smem = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   const int part_bytes = p.ngroups * 4 * p.gsize * 8;
+  p.sel_bytes = a.z == nullptr ? a.r * kUnit * 2 + a.r * 2 : 0;
   // deepest Bf and base rings that fit, favouring at least 4 base slots
   const int choices[][2] = {{6, 4}, {4, 4}, {6, 3}, {4, 3}, {4, 2}, {3, 2}, {2, 2}};
   size_t smem = 0;
   for (const auto& c : choices) {
-    const size_t need = make_layout(c[0], p.image_stride, c[1], part_bytes).total + 1024;
+    const size_t need = make_layout(c[0], p.image_stride, c[1], part_bytes, p.sel_bytes).total + 1024;
     if (static_cast<int>(need) <= max_smem) {
       p.nbf = c[0];
       p.nbs = c[1];
@@ -986,16 +977,7 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
   if (smem == 0) return cudaErrorInvalidConfiguration;
 
   CUtensorMap tm_bf, tm_base, tm_z;
-  {
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.V), static_cast<cuuint64_t>(a.r)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.V) * 2};
-    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kKStage)};
-    cuuint32_t es[2] = {1, 1};
-    if (enc(&tm_bf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.Bf), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
-  }
+  if (!encode_bf_tiles(&tm_bf, a.Bf, a.V, a.r)) return cudaErrorInvalidValue;
   auto enc3 = [&](CUtensorMap* tm, const float* ptr) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.V), static_cast<cuuint64_t>(a.K),
                           static_cast<cuuint64_t>(a.B)};
@@ -1006,11 +988,17 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   };
-  if (!enc3(&tm_base, a.base) || !enc3(&tm_z, a.z)) return cudaErrorInvalidValue;
+  // variant B writes no z: its map (never used) describes the base logits
+  if (!enc3(&tm_base, a.base) || !enc3(&tm_z, a.z != nullptr ? a.z : a.base)) return cudaErrorInvalidValue;
 
-  // the Markov head's kernel carries no code of the RNN head
-  const void* fn = a.W != nullptr ? reinterpret_cast<const void*>(&draft_tc_kernel<true>)
-                                  : reinterpret_cast<const void*>(&draft_tc_kernel<false>);
+  // the Markov head's kernel carries no code of the RNN head, and variant A's
+  // none of variant B's
+  const bool store_z = a.z != nullptr;
+  const void* fn = a.W != nullptr
+                       ? (store_z ? reinterpret_cast<const void*>(&draft_tc_kernel<true, true>)
+                                  : reinterpret_cast<const void*>(&draft_tc_kernel<true, false>))
+                       : (store_z ? reinterpret_cast<const void*>(&draft_tc_kernel<false, true>)
+                                  : reinterpret_cast<const void*>(&draft_tc_kernel<false, false>));
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;

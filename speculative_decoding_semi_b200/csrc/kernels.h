@@ -27,12 +27,21 @@ struct DraftArgs {
   float* part_m;    // [B][G]
   double* part_S;   // [B][G]
   const void* W;    // RNN head's recurrent weight [r,r] (bf16), or null for the Markov head
+  uint16_t* op_rows;  // variant B (z == null): [B,K,r] bf16 operand row of every position
 };
 
 struct VerifyArgs {
   const float* target;
   const int64_t* row_start;
-  const float* z;
+  const float* z;             // variant A: the draft logits; null in variant B
+  // variant B: z of a rejected row is recomputed as base + op_rows . Bf
+  const float* base;          // [B,K,V]
+  const uint16_t* op_rows;    // [B,K,r] bf16 bits
+  const void* Bf;             // [r,V] bf16
+  int r;
+  double* res_unit;           // scratch [V/32][B]: residual sums over 32-row units
+  double* res_part;           // scratch [B][grid]: residual sums over each CTA's slice
+  uint8_t* res_image;         // scratch: the residual groups' operand rows in the MMA's B layout
   const double* lse_q;
   const float* q_tok;
   const int32_t* tokens;

@@ -46,114 +46,14 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "verify_common.cuh"
 
 namespace dspark {
 
 namespace {
 
 using namespace sm100;
-
-constexpr int kSeg = 1024;                // row-pass segment: 32 lanes x 8 float4
-constexpr int kRSeg = 512;                // residual segment: 32 lanes x 4 float4
-constexpr int kCons = 8;                  // consumer warps per group (one segment each)
-constexpr int kGroups = 2;                // consumer groups, taking alternate stages
-constexpr int kProdWarp = kCons * kGroups;
-constexpr int kWarps = kProdWarp + 4;     // + producer + three more for the warp-per-unit phases
-constexpr int kThreads = kWarps * 32;
-constexpr int kRowItem = kCons * kSeg;    // logits per row item
-constexpr int kResItem = kCons * kRSeg;   // logits (and z values) per residual item
-constexpr int kStageBytes = kRowItem * 4;
-constexpr int kStages = 6;
-constexpr int kPlanThreads = 1024;
-constexpr int kRegSeg = 8;                // segment values per lane held in registers (nseg <= 256)
-constexpr double kSumLo = 1e-20, kSumHi = 1e30;
-constexpr float kLog2e = 1.44269504088896340736f;  // log2(e)
-constexpr double kLog2eD = 1.44269504088896340736;
-
-enum : int { kItemRow = 0, kItemRes = 1, kItemExit = 2 };
-// kCtlBar..kCtlBar+3: barrier counters
-enum : int { kCtlRows = 0, kCtlListed = 1, kCtlBar = 2, kCtlBonus = 6, kCtlCount = 8 };
-
-// One target row of the compact numbering.
-struct RowInfo {
-  int brl;        // b | rho << 16 | L_b << 22
-  int tok;        // drafted token tested at this row, -1 at the last row or if invalid
-  long long row;  // row index into the target logits
-};
-
-struct Desc {
-  int type, b, R, g;     // request, compact row, item index
-  int n, tok, pad0, pad1;  // logits in the item; drafted token (row items)
-  float shift[4], f[4];  // residual: per 1024-segment base-2 shift and p factor
-  float mq, fq, pad2[2];  // residual: q = 2^(z log2 e - mq) * fq
-};
-
-struct RowStat {
-  double M, W;  // base-2 largest shift, sum of 2^(x log2 e - M)
-};
-struct ResDec {
-  int acc, R;
-  long long row;  // target row of the rejection
-  float mq, fq;
-};
-
-struct Ws {
-  RowInfo* rowinfo;  // [B*(K+1)]
-  int* rowbase;      // [B] compact index of row 0, -1 for an invalid request
-  unsigned* ctl;     // counters, cleared by the plan kernel
-  float* part_m;     // [B*(K+1)][nseg] segment base-2 shift h
-  double* part_S;    // [B*(K+1)][nseg] segment sum of 2^(x log2 e - h)
-  float* x_tok;      // [B*(K+1)] logit at the drafted token (-inf if none)
-  RowStat* rstat;    // [B*(K+1)]
-  int* accepted;     // [B*(K+1)] accept test of the row's draft
-  ResDec* dec;       // [B]
-  float2* resfac;    // [B][nseg] residual (shift, p factor) per 1024-segment
-  int* list;         // [B] requests with a residual pass
-  int* blist;        // [B] requests whose drafts were all accepted (bonus draw)
-  double* seg_w;     // [B][nrseg] residual segment sums
-};
-
-struct Params {
-  VerifyArgs a;
-  Ws w;
-  int nseg, nrseg, ngrp, nrgrp;
-};
-
-// ------------------------------------------------------------ weights
-// The fp32 weights of the target distribution p and of the residual
-// max(0, p - q); explicit rounding intrinsics keep every site bit-identical.
-__device__ __forceinline__ float p_w(float x, float h) { return exp2f(__fmaf_rn(x, kLog2e, -h)); }
-__device__ __forceinline__ float res_w(float x, float z, float h, float f, float mq, float fq) {
-  const float p = __fmul_rn(exp2f(__fmaf_rn(x, kLog2e, -h)), f);
-  const float q = __fmul_rn(exp2f(__fmaf_rn(z, kLog2e, -mq)), fq);
-  const float d = __fsub_rn(p, q);
-  return d > 0.f ? d : 0.f;
-}
-__device__ __forceinline__ float group4(float w0, float w1, float w2, float w3) {
-  return __fadd_rn(__fadd_rn(__fadd_rn(w0, w1), w2), w3);
-}
-// 2^(h - M): the scale of a segment with base-2 shift h in a row whose largest
-// shift is M (exactly 1 in the common case h == M). The rare exponential is
-// kept out of line, so the common path carries neither its instructions nor
-// their evaluation.
-__device__ __noinline__ double exp2_rare(double x) { return exp2(x); }
-__device__ __forceinline__ double seg_scale(float h, double M) {
-  if (static_cast<double>(h) == M) return 1.0;
-  return exp2_rare(static_cast<double>(h) - M);
-}
-// (shift, factor) of a 1024-segment in the residual: p = 2^(x log2 e - h) * f.
-__device__ __forceinline__ float2 res_factor(float h, double M, double W) {
-  if (h == -INFINITY) return make_float2(0.f, 0.f);
-  return make_float2(h, static_cast<float>(seg_scale(h, M) / W));
-}
-// q = exp(z - lse) = 2^(z log2 e - mq) * fq with mq = fp32(lse log2 e).
-__device__ __forceinline__ void q_factor(double lse, float* mq, float* fq) {
-  const double c = lse * kLog2eD;
-  *mq = static_cast<float>(c);
-  *fq = static_cast<float>(exp2(static_cast<double>(*mq) - c));
-}
-
-__device__ __forceinline__ float4 neg_inf4() { return make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY); }
+using namespace vfy;
 
 // ------------------------------------------------------------ plan kernel
 __device__ int block_exscan_int(int v, int* total, int* red) {
@@ -232,150 +132,6 @@ __global__ void __launch_bounds__(kPlanThreads) verify_plan_kernel(Params p) {
   if (threadIdx.x < kCtlCount) p.w.ctl[threadIdx.x] = threadIdx.x == kCtlRows ? static_cast<unsigned>(carry) : 0u;
 }
 
-// ------------------------------------------------------ warp-level helpers
-// Inverse CDF over nseg segment weights, one warp; lane l owns the segments
-// [l per, l per + per). raw(q) loads what segment q's weight needs and
-// value(raw) computes the weight (the same value whenever called); the N <=
-// per-lane raw values are loaded before any is used, so their loads issue
-// together. Returns the first segment whose inclusive running sum exceeds
-// u * total with a positive weight, else (rounding) the last positive one,
-// with *rem = u * total minus the weight before it; -1 if total <= 0.
-template <int N, class Raw, class Value>
-__device__ int pick_segment_n(int nseg, float u, int lane, Raw raw, Value value, double* rem) {
-  const int per = (nseg + 31) / 32;
-  const int lo = min(nseg, lane * per), hi = min(nseg, lo + per);
-  using T = decltype(raw(0));
-  T rv[N];
-#pragma unroll
-  for (int i = 0; i < N; ++i) rv[i] = raw(min(lo + i, nseg - 1));  // clamped: always a valid address
-  double wv[N];
-  double local = 0.0;
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    wv[i] = lo + i < hi ? value(rv[i]) : 0.0;
-    local += wv[i];
-  }
-  const double inc = warp_inclusive_scan(local);
-  double ex = __shfl_up_sync(0xffffffffu, inc, 1);
-  if (lane == 0) ex = 0.0;
-  const double total = __shfl_sync(0xffffffffu, inc, 31);
-  if (!(total > 0.0)) return -1;
-  const double thr = static_cast<double>(u) * total;
-  int cand = INT_MAX, lastq = -1;
-  double cand_ex = 0.0, last_ex = 0.0, c = ex;
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const double v = wv[i];
-    if (v > 0.0) {
-      if (cand == INT_MAX && c + v > thr) {
-        cand = lo + i;
-        cand_ex = c;
-      }
-      lastq = lo + i;
-      last_ex = c;
-    }
-    c += v;
-  }
-  int seg = warp_min_int(cand);
-  double seg_ex;
-  if (seg != INT_MAX) {
-    seg_ex = __shfl_sync(0xffffffffu, cand_ex, seg / per);
-  } else {
-    seg = warp_max_int(lastq);
-    if (seg < 0) return -1;
-    seg_ex = __shfl_sync(0xffffffffu, last_ex, seg / per);
-  }
-  *rem = thr - seg_ex;
-  return seg;
-}
-
-// The same for any nseg: the smallest register block that holds per, or a
-// plain loop beyond 32 segments per lane.
-template <class Raw, class Value>
-__device__ int pick_segment(int nseg, float u, int lane, Raw raw, Value value, double* rem) {
-  const int per = (nseg + 31) / 32;
-  if (per <= 4) return pick_segment_n<4>(nseg, u, lane, raw, value, rem);
-  if (per <= 8) return pick_segment_n<8>(nseg, u, lane, raw, value, rem);
-  if (per <= 16) return pick_segment_n<16>(nseg, u, lane, raw, value, rem);
-  const int lo = min(nseg, lane * per), hi = min(nseg, lo + per);
-  double local = 0.0;
-  for (int q = lo; q < hi; ++q) local += value(raw(q));
-  const double inc = warp_inclusive_scan(local);
-  double ex = __shfl_up_sync(0xffffffffu, inc, 1);
-  if (lane == 0) ex = 0.0;
-  const double total = __shfl_sync(0xffffffffu, inc, 31);
-  if (!(total > 0.0)) return -1;
-  const double thr = static_cast<double>(u) * total;
-  int cand = INT_MAX, lastq = -1;
-  double cand_ex = 0.0, last_ex = 0.0, c = ex;
-  for (int q = lo; q < hi; ++q) {
-    const double v = value(raw(q));
-    if (v > 0.0) {
-      if (cand == INT_MAX && c + v > thr) {
-        cand = q;
-        cand_ex = c;
-      }
-      lastq = q;
-      last_ex = c;
-    }
-    c += v;
-  }
-  int seg = warp_min_int(cand);
-  double seg_ex;
-  if (seg != INT_MAX) {
-    seg_ex = __shfl_sync(0xffffffffu, cand_ex, seg / per);
-  } else {
-    seg = warp_max_int(lastq);
-    if (seg < 0) return -1;
-    seg_ex = __shfl_sync(0xffffffffu, last_ex, seg / per);
-  }
-  *rem = thr - seg_ex;
-  return seg;
-}
-
-// First element of a run of n <= 32 * E elements whose running sum of
-// weights exceeds R with a positive weight, or -1 (then *last = the last
-// positive one); one warp. Lane l owns elements [E l, E l + E): w[] holds
-// their fp32 weights (zero past n). Four consecutive weights form one fp32
-// group exactly as in the segment sums; the groups accumulate in fp64, one
-// warp-wide scan over the lanes' totals, then a search inside one lane.
-template <int E>
-__device__ int rescan(int n, int lane, double R, const float (&w)[E], int* last) {
-  float c[E];  // inclusive fp32 sums within each group of four
-  double lsum = 0.0;
-#pragma unroll
-  for (int k = 0; k < E / 4; ++k) {
-    c[4 * k] = w[4 * k];
-    c[4 * k + 1] = __fadd_rn(c[4 * k], w[4 * k + 1]);
-    c[4 * k + 2] = __fadd_rn(c[4 * k + 1], w[4 * k + 2]);
-    c[4 * k + 3] = __fadd_rn(c[4 * k + 2], w[4 * k + 3]);
-    lsum += static_cast<double>(c[4 * k + 3]);
-  }
-  const double inc = warp_inclusive_scan(lsum);
-  double before = __shfl_up_sync(0xffffffffu, inc, 1);
-  if (lane == 0) before = 0.0;
-  int hit = -1, lp = -1;
-  if (before + lsum > R) {
-#pragma unroll
-    for (int k = 0; k < E / 4; ++k) {
-      if (hit < 0) {
-#pragma unroll
-        for (int j = 3; j >= 0; --j)
-          if (w[4 * k + j] > 0.f && before + static_cast<double>(c[4 * k + j]) > R) hit = 4 * k + j;
-        before += static_cast<double>(c[4 * k + 3]);
-      }
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < E; ++e)
-    if (w[e] > 0.f) lp = E * lane + e;
-  *last = warp_max_int(lp);
-  const unsigned hits = __ballot_sync(0xffffffffu, hit >= 0);
-  if (!hits) return -1;
-  const int hl = __ffs(hits) - 1;
-  return E * hl + __shfl_sync(0xffffffffu, hit, hl);
-}
-
 // Phase 2, one warp: (M, W) of compact row R from its segment partials, and
 // the accept test of the row's draft.
 __device__ void row_stats(const Params& P, int R, int lane) {
@@ -426,58 +182,6 @@ __device__ void row_stats(const Params& P, int R, int lane) {
   }
 }
 
-// Draw from p of compact row R (the bonus row, or a rejected row whose
-// residual vanished) with the row pass's segment sums; one warp. With `warm`
-// set it runs its whole path on whatever the arrays hold, to load its code
-// into the SM's instruction cache ahead of the phase that needs it.
-__device__ __noinline__ int sample_p(const Params& P, int R, float u, int lane, bool warm = false) {
-  const VerifyArgs& a = P.a;
-  const float* pm = P.w.part_m + static_cast<long long>(R) * P.nseg;
-  const double* pS = P.w.part_S + static_cast<long long>(R) * P.nseg;
-  const double M = __ldcg(&P.w.rstat[R].M);
-  const long long row = P.w.rowinfo[R].row;
-  // segment weights S 2^(h - M): the row's total W scales them all alike and
-  // cancels in the inverse CDF
-  double rem = 0.0;
-  const int seg = pick_segment(
-      P.nseg, u, lane, [&](int q) { return make_double2(__ldcg(pS + q), static_cast<double>(__ldcg(pm + q))); },
-      [&](double2 r) { return r.x > 0.0 ? __dmul_rn(r.x, seg_scale(static_cast<float>(r.y), M)) : 0.0; }, &rem);
-  if (seg < 0 && !warm) return 0;  // no positive weight: degenerate row
-  const int sg = max(seg, 0);
-  const float m_s = __ldcg(pm + sg);
-  const double Rs = rem / seg_scale(m_s, M);
-  const float* x = a.target + row * a.V + static_cast<long long>(sg) * kSeg;
-  const int n = min(kSeg, a.V - sg * kSeg);
-  constexpr int E = kSeg / 32;
-  float w[E];
-#pragma unroll
-  for (int k = 0; k < E / 4; ++k) {
-    const int e = E * lane + 4 * k;
-    const float4 v = e < n ? __ldcg(reinterpret_cast<const float4*>(x + e)) : neg_inf4();
-    w[4 * k] = p_w(v.x, m_s);
-    w[4 * k + 1] = p_w(v.y, m_s);
-    w[4 * k + 2] = p_w(v.z, m_s);
-    w[4 * k + 3] = p_w(v.w, m_s);
-  }
-  int last = -1;
-  int k = rescan<E>(n, lane, Rs, w, &last);
-  if (k < 0) k = max(last, 0);
-  return sg * kSeg + k;
-}
-
-// Emits request b's accepted drafts and the drawn token.
-__device__ void write_output(const Params& P, int b, int acc, int tok, int lane) {
-  const VerifyArgs& a = P.a;
-  int32_t* out = a.out_tokens + static_cast<long long>(b) * (a.K + 1);
-  // j = 32 (K = 32 only) is never an accepted draft, since acc <= K
-  for (int j = lane; j <= a.K; j += 32)
-    out[j] = j < acc ? a.tokens[static_cast<long long>(b) * a.K + j] : (j == acc ? tok : -1);
-  if (lane == 0) {
-    a.accepted[b] = acc;
-    a.n_out[b] = acc + 1;
-  }
-}
-
 // Phase 3, one warp: request b's first rejection; a place in the list of
 // bonus draws, or the residual pass's inputs and a place in its list.
 // With `warm` set it writes nothing: it runs once during phase 1 to load its
@@ -499,6 +203,35 @@ __device__ __noinline__ void decide(const Params& P, int b, int lane, bool warm 
     return;
   }
   const double M = __ldcg(&P.w.rstat[R].M), W = __ldcg(&P.w.rstat[R].W);
+  if (P.recompute) {
+    // variant B: the residual kernel weighs the row with its own (shift,
+    // factor); its operand row goes to the group's image in the MMA's B
+    // layout (K-major, 128-byte swizzle, blocks of 64 rank values gsize rows apart)
+    if (warm) return;
+    unsigned e = 0;
+    if (lane == 0) {
+      ResSlot s{};
+      s.b = b;
+      s.acc = acc;
+      s.row = P.w.rowinfo[R].row;
+      s.brow = b * a.K + acc;
+      s.R = R;
+      q_factor(a.lse_q[static_cast<long long>(b) * a.K + acc], &s.mq, &s.fq);
+      p_factor(M, W, &s.mp, &s.fp);
+      e = atomicAdd(P.w.ctl + kCtlListed, 1u);
+      P.w.slots[e] = s;
+      P.w.list[e] = b;
+    }
+    e = __shfl_sync(0xffffffffu, e, 0);
+    const int gs = P.res_gsize, gr = static_cast<int>(e) / gs, n = static_cast<int>(e) % gs;
+    if (lane < a.r / 8) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.op_rows + (static_cast<long long>(b) * a.K + acc) * a.r) + lane);
+      const int kb = lane >> 3, c = lane & 7;
+      *reinterpret_cast<uint4*>(a.res_image + static_cast<long long>(gr) * gs * a.r * 2 + kb * (gs * 128) + n * 128 +
+                                ((c ^ (n & 7)) << 4)) = v;
+    }
+    return;
+  }
   const float* pm = P.w.part_m + static_cast<long long>(R) * P.nseg;
   float2* rf = P.w.resfac + static_cast<long long>(b) * P.nseg;
   for (int q0 = 0; q0 < P.nseg; q0 += 32 * kRegSeg) {
@@ -770,7 +503,10 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
         ds.tok = ri.tok;
         const uint32_t bytes = static_cast<uint32_t>(n) * 4u;
         mbar_arrive_expect_tx(full, bytes);
-        bulk_load(dst, a.target + ri.row * a.V + v0, bytes, full);
+        // variant B: evict-first, so that the draft's Bf (evict-last) stays in
+        // L2 for the residual kernel that follows
+        if (P.recompute) bulk_load_hint(dst, a.target + ri.row * a.V + v0, bytes, full, policy_evict_first());
+        else bulk_load(dst, a.target + ri.row * a.V + v0, bytes, full);
       },
       [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_row(P, ds, stage, empty, w, lane); });
   // the spare warps run the later phases' code once while the rows stream, so
@@ -778,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
   if (warp > kProdWarp && n_rows > 0) {
     int r = 0;
     if (warp == kProdWarp + 1) r = sample_p(P, 0, 0.5f, lane, true);
-    if (warp == kProdWarp + 2) {
+    if (warp == kProdWarp + 2 && !P.recompute) {
       ResDec d{};
       d.row = P.w.rowinfo[0].row;
       r = residual_token(P, 0, d, 0.5f, lane, true);
@@ -801,57 +537,70 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
     for (int b = gw; b < a.B; b += NW) decide(P, b, lane);
   ok = ok && grid_barrier(P, 2, &s_flag);
 
-  // ---- phase 4: residual segment sums of the listed requests
-  const int n_listed = ok ? static_cast<int>(__ldcg(P.w.ctl + kCtlListed)) : 0;
-  if (ok) {
-    const uint64_t pol_first = policy_evict_first();
-    ok = stream(
-        static_cast<long long>(n_listed) * P.nrgrp,
-        [&](long long item, Desc& ds, float* dst, uint64_t* full) {
-          const int e = static_cast<int>(item / P.nrgrp), g = static_cast<int>(item % P.nrgrp);
-          const int b = __ldcg(P.w.list + e);
-          const ResDec d = P.w.dec[b];
-          const int v0 = g * kResItem, n = min(kResItem, a.V - v0);
-          ds.type = kItemRes;
-          ds.b = b;
-          ds.R = d.R;
-          ds.g = g;
-          ds.n = n;
-          ds.tok = -1;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int q = g * 4 + i;
-            const float2 f =
-                q < P.nseg ? __ldcg(P.w.resfac + static_cast<long long>(b) * P.nseg + q) : make_float2(0.f, 0.f);
-            ds.shift[i] = f.x;
-            ds.f[i] = f.y;
-          }
-          ds.mq = d.mq;
-          ds.fq = d.fq;
-          const uint32_t bytes = static_cast<uint32_t>(n) * 4u;
-          mbar_arrive_expect_tx(full, 2u * bytes);
-          bulk_load(dst, a.target + d.row * a.V + v0, bytes, full);
-          bulk_load_hint(dst + kResItem, a.z + (static_cast<long long>(b) * a.K + d.acc) * a.V + v0, bytes, full,
-                         pol_first);
-        },
-        [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_res(P, ds, stage, empty, w, lane); });
-    // meanwhile the warps outside the stream make the bonus draws
-    if (warp > kProdWarp) {
+  // variant B: the bonus draws, one warp per request; the residual kernel
+  // that follows does the rest
+  if (P.recompute) {
+    if (ok) {
       const int n_bonus = static_cast<int>(__ldcg(P.w.ctl + kCtlBonus));
-      const int nsw = (kWarps - kProdWarp - 1) * G;
-      for (int e = (warp - kProdWarp - 1) * G + c; e < n_bonus; e += nsw) {
+      for (int e = gw; e < n_bonus; e += NW) {
         const int b = __ldcg(P.w.blist + e);
         const int L = a.verify_len[b];
-        const int tok = sample_p(P, P.w.rowbase[b] + L, a.u_resample[b], lane);
-        write_output(P, b, L, tok, lane);
+        write_output(P, b, L, sample_p(P, P.w.rowbase[b] + L, a.u_resample[b], lane), lane);
       }
     }
-    ok = __syncthreads_and(ok) && grid_barrier(P, 3, &s_flag);
-  }
+  } else {
+    // ---- phase 4: residual segment sums of the listed requests
+    const int n_listed = ok ? static_cast<int>(__ldcg(P.w.ctl + kCtlListed)) : 0;
+    if (ok) {
+      const uint64_t pol_first = policy_evict_first();
+      ok = stream(
+          static_cast<long long>(n_listed) * P.nrgrp,
+          [&](long long item, Desc& ds, float* dst, uint64_t* full) {
+            const int e = static_cast<int>(item / P.nrgrp), g = static_cast<int>(item % P.nrgrp);
+            const int b = __ldcg(P.w.list + e);
+            const ResDec d = P.w.dec[b];
+            const int v0 = g * kResItem, n = min(kResItem, a.V - v0);
+            ds.type = kItemRes;
+            ds.b = b;
+            ds.R = d.R;
+            ds.g = g;
+            ds.n = n;
+            ds.tok = -1;
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int q = g * 4 + i;
+              const float2 f =
+                  q < P.nseg ? __ldcg(P.w.resfac + static_cast<long long>(b) * P.nseg + q) : make_float2(0.f, 0.f);
+              ds.shift[i] = f.x;
+              ds.f[i] = f.y;
+            }
+            ds.mq = d.mq;
+            ds.fq = d.fq;
+            const uint32_t bytes = static_cast<uint32_t>(n) * 4u;
+            mbar_arrive_expect_tx(full, 2u * bytes);
+            bulk_load(dst, a.target + d.row * a.V + v0, bytes, full);
+            bulk_load_hint(dst + kResItem, a.z + (static_cast<long long>(b) * a.K + d.acc) * a.V + v0, bytes, full,
+                           pol_first);
+          },
+          [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_res(P, ds, stage, empty, w, lane); });
+      // meanwhile the warps outside the stream make the bonus draws
+      if (warp > kProdWarp) {
+        const int n_bonus = static_cast<int>(__ldcg(P.w.ctl + kCtlBonus));
+        const int nsw = (kWarps - kProdWarp - 1) * G;
+        for (int e = (warp - kProdWarp - 1) * G + c; e < n_bonus; e += nsw) {
+          const int b = __ldcg(P.w.blist + e);
+          const int L = a.verify_len[b];
+          const int tok = sample_p(P, P.w.rowbase[b] + L, a.u_resample[b], lane);
+          write_output(P, b, L, tok, lane);
+        }
+      }
+      ok = __syncthreads_and(ok) && grid_barrier(P, 3, &s_flag);
+    }
 
-  // ---- phase 5: resampled tokens
-  if (ok)
-    for (int e = gw; e < n_listed; e += NW) resample(P, __ldcg(P.w.list + e), lane);
+    // ---- phase 5: resampled tokens
+    if (ok)
+      for (int e = gw; e < n_listed; e += NW) resample(P, __ldcg(P.w.list + e), lane);
+  }
 
   // copies still in flight (after an abort) land before the CTA exits
   __syncthreads();
@@ -861,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
 }
 
 struct Layout {
-  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, blist, seg_w, total;
+  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, blist, seg_w, slots, total;
 };
 
 Layout verify_layout(int B, int K, int V) {
@@ -887,6 +636,7 @@ Layout verify_layout(int B, int K, int V) {
   L.list = take(nb * sizeof(int));
   L.blist = take(nb * sizeof(int));
   L.seg_w = take(nb * nrseg * sizeof(double));
+  L.slots = take(nb * sizeof(ResSlot));
   L.total = off;
   return L;
 }
@@ -916,6 +666,9 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
   P.w.list = reinterpret_cast<int*>(region + L.list);
   P.w.blist = reinterpret_cast<int*>(region + L.blist);
   P.w.seg_w = reinterpret_cast<double*>(region + L.seg_w);
+  P.w.slots = reinterpret_cast<ResSlot*>(region + L.slots);
+  P.recompute = a.z == nullptr ? 1 : 0;
+  P.res_gsize = residual_group_size(a.B);
 
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
@@ -965,7 +718,8 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, verify_kernel, P);
   }
-  return e;
+  if (e != cudaSuccess || !P.recompute) return e;
+  return launch_residual_tc(P, stream);
 }
 
 }  // namespace dspark

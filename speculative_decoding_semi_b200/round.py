@@ -12,8 +12,9 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from .binding import (dspark_advance_anchor, dspark_calibrate, dspark_markov_draft, dspark_rnn_draft, dspark_schedule,
-                      dspark_verify, dspark_workspace_bytes, dspark_workspace_init)
+from .binding import (dspark_advance_anchor, dspark_calibrate, dspark_markov_draft, dspark_markov_draft_b,
+                      dspark_rnn_draft, dspark_rnn_draft_b, dspark_schedule, dspark_verify, dspark_verify_b,
+                      dspark_workspace_bytes, dspark_workspace_init)
 
 
 def to_device(inputs: dict, device="cuda") -> dict:
@@ -34,13 +35,20 @@ def to_device(inputs: dict, device="cuda") -> dict:
 
 
 class RoundBuffers:
-    def __init__(self, B: int, K: int, V: int, r: int, device="cuda"):
-        self.B, self.K, self.V, self.r = B, K, V, r
+    """Variant "a" stores the draft logits z [B,K,V]; variant "b" stores the
+    operand rows op_rows [B,K,r] (bf16) instead and verification recomputes
+    the rejected row of z."""
+
+    def __init__(self, B: int, K: int, V: int, r: int, device="cuda", variant: str = "a"):
+        if variant not in ("a", "b"):
+            raise ValueError("variant must be 'a' or 'b'")
+        self.B, self.K, self.V, self.r, self.variant = B, K, V, r, variant
         i32, f32, f64 = torch.int32, torch.float32, torch.float64
         self.draft_tokens = torch.empty(B, K, dtype=i32, device=device)
         self.q_tok = torch.empty(B, K, dtype=f32, device=device)
         self.lse_q = torch.empty(B, K, dtype=f64, device=device)
-        self.z = torch.empty(B, K, V, dtype=f32, device=device)
+        self.z = torch.empty(B, K, V, dtype=f32, device=device) if variant == "a" else None
+        self.op_rows = torch.empty(B, K, r, dtype=torch.bfloat16, device=device) if variant == "b" else None
         self.verify_len = torch.empty(B, dtype=i32, device=device)
         self.survival = torch.empty(B, K, dtype=f32, device=device)
         self.row_start = torch.empty(B, dtype=torch.int64, device=device)
@@ -52,30 +60,42 @@ class RoundBuffers:
         dspark_workspace_init(self.workspace)
 
 
-def draft(d: dict, bufs: RoundBuffers, stream=None):
-    """The Markov head, or the RNN head when d holds its recurrent weight "W"."""
-    if d.get("W") is not None:
-        dspark_rnn_draft(d["base"], d["A"], d["W"], d["Bf"], d["anchor"], d["u_draft"], bufs.draft_tokens, bufs.q_tok,
-                         bufs.lse_q, bufs.z, bufs.workspace, stream)
+def draft(d: dict, bufs: RoundBuffers, stream=None, anchor=None):
+    """The Markov head, or the RNN head when d holds its recurrent weight "W";
+    `anchor` overrides d["anchor"]."""
+    anchor = d["anchor"] if anchor is None else anchor
+    out = (bufs.draft_tokens, bufs.q_tok, bufs.lse_q)
+    if bufs.variant == "b":
+        if d.get("W") is not None:
+            dspark_rnn_draft_b(d["base"], d["A"], d["W"], d["Bf"], anchor, d["u_draft"], *out, bufs.op_rows,
+                               bufs.workspace, stream)
+        else:
+            dspark_markov_draft_b(d["base"], d["A"], d["Bf"], anchor, d["u_draft"], *out, bufs.op_rows,
+                                  bufs.workspace, stream)
+    elif d.get("W") is not None:
+        dspark_rnn_draft(d["base"], d["A"], d["W"], d["Bf"], anchor, d["u_draft"], *out, bufs.z, bufs.workspace,
+                         stream)
     else:
-        dspark_markov_draft(d["base"], d["A"], d["Bf"], d["anchor"], d["u_draft"], bufs.draft_tokens, bufs.q_tok,
-                            bufs.lse_q, bufs.z, bufs.workspace, stream)
+        dspark_markov_draft(d["base"], d["A"], d["Bf"], anchor, d["u_draft"], *out, bufs.z, bufs.workspace, stream)
 
 
-def schedule(d: dict, bufs: RoundBuffers, stream=None):
-    dspark_schedule(d["conf"], d["temps"], d["profile"], bufs.verify_len, bufs.survival, bufs.row_start,
-                    bufs.n_tokens, bufs.workspace, stream)
+def schedule(d: dict, bufs: RoundBuffers, stream=None, temps=None):
+    dspark_schedule(d["conf"], d["temps"] if temps is None else temps, d["profile"], bufs.verify_len, bufs.survival,
+                    bufs.row_start, bufs.n_tokens, bufs.workspace, stream)
 
 
 def verify(d: dict, bufs: RoundBuffers, target=None, row_start=None, verify_len=None, stream=None):
     """Verify against `target` rows addressed by `row_start` (default: the dense
     [B,K+1,V] target of `d`, row_start[b] = b*(K+1))."""
-    dspark_verify(d["target"] if target is None else target,
-                  d["row_start_dense"] if row_start is None else row_start,
-                  bufs.z, bufs.lse_q, bufs.q_tok, bufs.draft_tokens,
-                  bufs.verify_len if verify_len is None else verify_len,
-                  d["u_accept"], d["u_resample"], bufs.accepted, bufs.out_tokens, bufs.n_out,
-                  bufs.workspace, stream)
+    target = d["target"] if target is None else target
+    row_start = d["row_start_dense"] if row_start is None else row_start
+    verify_len = bufs.verify_len if verify_len is None else verify_len
+    tail = (bufs.lse_q, bufs.q_tok, bufs.draft_tokens, verify_len, d["u_accept"], d["u_resample"], bufs.accepted,
+            bufs.out_tokens, bufs.n_out, bufs.workspace, stream)
+    if bufs.variant == "b":
+        dspark_verify_b(target, row_start, d["base"], bufs.op_rows, d["Bf"], *tail)
+    else:
+        dspark_verify(target, row_start, bufs.z, *tail)
 
 
 def run_round(d: dict, bufs: RoundBuffers, stream=None):
@@ -126,13 +146,9 @@ def run_rounds(inputs: list, bufs: RoundBuffers, state: RoundState, rounds: int,
             if record:
                 hist["anchor"][r].copy_(state.anchor, non_blocking=True)
                 hist["temps"][r].copy_(state.temps, non_blocking=True)
-            dspark_markov_draft(d["base"], d["A"], d["Bf"], state.anchor, d["u_draft"], bufs.draft_tokens,
-                                bufs.q_tok, bufs.lse_q, bufs.z, bufs.workspace, s)
-            dspark_schedule(d["conf"], state.temps, d["profile"], bufs.verify_len, bufs.survival, bufs.row_start,
-                            bufs.n_tokens, bufs.workspace, s)
-            dspark_verify(d["target"], d["row_start_dense"], bufs.z, bufs.lse_q, bufs.q_tok, bufs.draft_tokens,
-                          bufs.verify_len, d["u_accept"], d["u_resample"], bufs.accepted, bufs.out_tokens, bufs.n_out,
-                          bufs.workspace, s)
+            draft(d, bufs, s, anchor=state.anchor)
+            schedule(d, bufs, s, temps=state.temps)
+            verify(d, bufs, stream=s)
             if record:
                 for name in HISTORY:
                     if name not in ("anchor", "temps"):

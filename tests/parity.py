@@ -177,16 +177,17 @@ def _full(vals, requests, B):
     return out
 
 
-def gpu_round(inp, requests=None, packed=False, bufs=None):
+def gpu_round(inp, requests=None, packed=False, bufs=None, variant="a"):
     """Run draft -> schedule -> verify through the library; numpy outputs.
-    `bufs` (optional) reuses the outputs and workspace of an earlier round."""
+    `bufs` (optional) reuses the outputs and workspace of an earlier round;
+    variant "b" stores no z (the draft returns the operand rows instead)."""
     from speculative_decoding_semi_b200 import round as rnd
 
     B, K, V = inp["base"].shape
     r = inp["A"].shape[1]
     d = rnd.to_device(inp)
     if bufs is None:
-        bufs = rnd.RoundBuffers(B, K, V, r)
+        bufs = rnd.RoundBuffers(B, K, V, r, variant=variant)
     rnd.draft(d, bufs)
     rnd.schedule(d, bufs)
     if packed:
@@ -201,11 +202,14 @@ def gpu_round(inp, requests=None, packed=False, bufs=None):
     st, detail = dspark_read_device_error(bufs.workspace)
     assert st == 0, (st, hex(detail))
     reqs = np.arange(B) if requests is None else np.asarray(requests)
-    ridx = torch.as_tensor(reqs, device=bufs.z.device)
+    ridx = torch.as_tensor(reqs, device=bufs.draft_tokens.device)
     take = lambda t: t.index_select(0, ridx).cpu().numpy()
+    keep_z = bufs.z is not None and len(reqs) * K * V <= 64 * 16 * 151936
     out = {
         "draft": {"tokens": take(bufs.draft_tokens), "q_tok": take(bufs.q_tok), "lse_q": take(bufs.lse_q),
-                  "z": take(bufs.z) if len(reqs) * K * V <= 64 * 16 * 151936 else None},
+                  "z": take(bufs.z) if keep_z else None,
+                  "op_rows": (take(bufs.op_rows.view(torch.int16)).view(np.uint16)
+                              if bufs.op_rows is not None else None)},
         "schedule": {"verify_len": bufs.verify_len.cpu().numpy(), "survival": bufs.survival.cpu().numpy(),
                      "row_start": bufs.row_start.cpu().numpy(), "n_tokens": bufs.n_tokens.cpu().numpy()[0]},
         "verify": {"accepted": take(bufs.accepted), "out_tokens": take(bufs.out_tokens), "n_out": take(bufs.n_out)},
@@ -221,10 +225,38 @@ def compare_round(inp, g, reqs, tally: Tally, check_z=True):
     compare_verify(inp, d, g["draft"], g["verify"], g["schedule"]["verify_len"], reqs, tally)
 
 
-def check_round(inp, requests=None, packed=False, tally: Tally | None = None, check_z=True, bufs=None):
+def check_op_rows(inp, gpu_draft, requests, tally: Tally):
+    """Variant B: the operand row of position i must be A[t_{i-1}] bit for bit
+    (t_{-1} the anchor) for the Markov head; for the RNN head the oracle's
+    state h_i (teacher-forced on the GPU's tokens) rounded to bf16, within one
+    bf16 step (the two fp64 states differ by rounding)."""
+    rows = gpu_draft["op_rows"]
+    toks = gpu_draft["tokens"].astype(np.int64)
+    anchor = np.asarray(inp["anchor"])[requests].astype(np.int64)
+    prev = np.concatenate([anchor[:, None], toks[:, :-1]], axis=1)
+    if inp.get("W") is None:
+        want = np.asarray(inp["A"])[prev]
+        bad = np.argwhere(np.any(rows != want, axis=-1))
+        if len(bad):
+            tally.failures.append(("op_rows", [tuple(int(x) for x in b) for b in bad[:5]]))
+        return
+    d = oracle.rnn_draft(inp["base"][requests], inp["A"], inp["W"], inp["Bf"], anchor, inp["u_draft"][requests],
+                         teacher=toks, keep_z=False)
+    want = oracle.round_to_bf16(d["h"])
+    got = synth.bf16_bits_to_f32(rows).astype(np.float64)
+    step = np.abs(want) * 2.0 ** -7 + 1e-40
+    err = np.abs(got - want) / step
+    if err.max() > 1.0 + 1e-9:
+        tally.failures.append(("op_rows rnn", float(err.max())))
+
+
+def check_round(inp, requests=None, packed=False, tally: Tally | None = None, check_z=True, bufs=None,
+                variant="a"):
     B = inp["base"].shape[0]
     reqs = np.arange(B) if requests is None else np.asarray(requests)
-    g = gpu_round(inp, reqs, packed=packed, bufs=bufs)
+    g = gpu_round(inp, reqs, packed=packed, bufs=bufs, variant=variant)
     t = Tally() if tally is None else tally
     compare_round(inp, g, reqs, t, check_z=check_z)
+    if g["draft"]["op_rows"] is not None:
+        check_op_rows(inp, g["draft"], reqs, t)
     return t, g

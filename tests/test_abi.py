@@ -70,3 +70,34 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert st == 1
     st = lib.dspark_workspace_init(nul, 1 << 20, None)
     assert st == 1
+
+
+def test_variant_b_shapes_rejected_before_launch(lib):
+    """Variant B runs on the tensor-core kernels only: other shapes return
+    DSPARK_ERR_UNSUPPORTED (2) before anything touches the GPU."""
+    P = ctypes.c_void_p
+    fake = P(4096)
+    ws = 1 << 40
+    # fp32 factors; r = 32; V % 32 != 0; B > 512
+    for dt, r, B, V in ((0, 64, 4, 1024), (1, 32, 4, 1024), (1, 64, 4, 1000), (1, 64, 513, 1024)):
+        st = lib.dspark_markov_draft_b(fake, fake, fake, dt, r, fake, fake, B, 4, V, fake, fake, fake, fake,
+                                       fake, ws, None)
+        assert st == 2, (dt, r, B, V)
+        st = lib.dspark_rnn_draft_b(fake, fake, fake, fake, dt, r, fake, fake, B, 4, V, fake, fake, fake, fake,
+                                    fake, ws, None)
+        assert st == 2, (dt, r, B, V)
+    for r, B, V in ((32, 4, 1024), (64, 4, 1000), (64, 513, 1024)):
+        st = lib.dspark_verify_b(fake, fake, fake, fake, fake, r, fake, fake, fake, fake, fake, fake, B, 4, V,
+                                 fake, fake, fake, fake, ws, None)
+        assert st == 2, (r, B, V)
+    # NULL operand rows / base are invalid arguments
+    st = lib.dspark_markov_draft_b(fake, fake, fake, 1, 64, fake, fake, 4, 4, 1024, fake, fake, fake, None,
+                                   fake, ws, None)
+    assert st == 1
+    st = lib.dspark_verify_b(fake, fake, None, fake, fake, 64, fake, fake, fake, fake, fake, fake, 4, 4, 1024,
+                             fake, fake, fake, fake, ws, None)
+    assert st == 1
+    # variant A entry points still need z
+    st = lib.dspark_markov_draft(fake, fake, fake, 1, 64, fake, fake, 4, 4, 1024, fake, fake, fake, None,
+                                 fake, ws, None)
+    assert st == 1
