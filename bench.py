@@ -172,18 +172,31 @@ def measured_traffic(workload: str) -> dict:
     return {k: v for k, v in tj.get("dram_bytes_per_launch", {}).items()}
 
 
-def draft_bytes(B, K, V, r, factor_bytes):
-    """Algorithmic HBM bytes of one draft launch: base read + z write + Bf once
-    + gathered A rows + per-position outputs."""
-    return B * K * V * 4 * 2 + r * V * factor_bytes + B * K * r * factor_bytes + B * K * (4 + 4 + 8 + 4)
+def draft_bytes(B, K, V, r, factor_bytes, variant="a"):
+    """Algorithmic HBM bytes of one draft launch: base read + z write (variant
+    A) or the operand rows (variant B) + Bf once + gathered A rows +
+    per-position outputs."""
+    out = B * K * V * 4 if variant == "a" else B * K * r * 2
+    return B * K * V * 4 + out + r * V * factor_bytes + B * K * r * factor_bytes + B * K * (4 + 4 + 8 + 4)
 
 
-def verify_bytes(V, K, verify_len, accepted):
+def verify_bytes(V, K, verify_len, accepted, r=256, factor_bytes=2, variant="a"):
     """Algorithmic HBM bytes of one verify call: every target row 0..L_b once,
-    plus the z row of each rejected request (the residual needs q there)."""
+    plus, for each rejected request, the z row (variant A) or the base row,
+    with Bf once and the operand rows, to recompute it (variant B)."""
     rows = int((verify_len + 1).sum())
     rejected = int((accepted < verify_len).sum())
-    return rows * V * 4 + rejected * V * 4
+    extra = 0 if variant == "a" or rejected == 0 else r * V * factor_bytes + rejected * r * 2
+    return rows * V * 4 + rejected * V * 4 + extra
+
+
+def round_variant(choice: str, B: int) -> str:
+    """Variant A stores z; variant B recomputes the rejected rows in verify.
+    B measured faster from B = 128 on (the z write grows with B; the
+    recompute's pass over Bf does not), A below that."""
+    if choice != "auto":
+        return choice
+    return "b" if B >= 128 else "a"
 
 
 def run_reference(args):
@@ -240,10 +253,12 @@ def run_gpu(args):
     inp = synth.make_round(w, seed=w.seed + rank)
     B, K, V, r = w.B, w.K, w.V, w.r
     d = rnd.to_device(inp)
-    bufs = rnd.RoundBuffers(B, K, V, r)
+    variant = round_variant(args.variant, B)
+    bufs = rnd.RoundBuffers(B, K, V, r, variant=variant)
     stream = torch.cuda.Stream()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-    launches_per_round = 1 + 2 + 2  # draft, schedule (rank, final), verify (plan, main)
+    # draft, schedule (rank, final), verify (plan, main), and variant B's residual kernel
+    launches_per_round = 1 + 2 + 2 + (1 if variant == "b" else 0)
 
     def one_round(ev=None):
         with torch.cuda.stream(stream):
@@ -292,15 +307,15 @@ def run_gpu(args):
     n_out = bufs.n_out.cpu().numpy()
     peaks = measured_peaks()
     fb = 2 if w.factor_dtype == "bf16" else 4
-    dbytes = draft_bytes(B, K, V, r, fb)
-    vbytes = verify_bytes(V, K, L, acc)
+    dbytes = draft_bytes(B, K, V, r, fb, variant)
+    vbytes = verify_bytes(V, K, L, acc, r, fb, variant)
     med = statistics.median
     draft_gbs = dbytes / (med(t_draft) * 1e-3) / 1e9
     verify_gbs = vbytes / (med(t_ver) * 1e-3) / 1e9
     round_gbs = (dbytes + vbytes) / (med(t_round) * 1e-3) / 1e9
     # the draft's floor if verify recomputed the rejected z rows instead of
     # reading them back (z never written): base read + Bf once + the rest
-    dbytes_b = dbytes - B * K * V * 4
+    dbytes_b = draft_bytes(B, K, V, r, fb, "b")
 
     # end to end through the public API with host buffers: copy this round's
     # inputs from pinned host memory, run the round, read the result back
@@ -341,19 +356,22 @@ def run_gpu(args):
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
         "dtype_detail": "fp32 logits, bf16 Markov factors with fp32 accumulation, fp64 vocabulary sums",
-        "data": "synthetic", "config": config_of(w),
+        "data": "synthetic", "config": dict(config_of(w), variant=variant),
         "tokens_per_s": value * float(n_out.sum()),
         "stages_ms_median": {"draft": med(t_draft), "schedule": med(t_sched), "verify": med(t_ver)},
         "draft_us_per_position": 1000.0 * med(t_draft) / K,
         "round_ms": {"median": med(t_round), "p10": float(np.percentile(t_round, 10)),
                      "p90": float(np.percentile(t_round, 90))},
-        "roofline": {"bound": "hbm", "kernel": "dspark_markov_draft", "achieved": draft_gbs,
+        "roofline": {"bound": "hbm", "kernel": "dspark_markov_draft" + ("_b" if variant == "b" else ""),
+                     "achieved": draft_gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": draft_gbs / peaks["hbm_gbs"],
-                     "traffic": traffic.get("draft_tc_kernel"), "algorithmic_bytes": dbytes,
+                     "traffic": traffic.get("draft_tc_kernel") if variant == "a" else None,
+                     "algorithmic_bytes": dbytes,
                      "peak_source": peaks["source"], "frac_nominal": draft_gbs / NOMINAL_HBM_GBS,
                      "frac_design_b_floor": dbytes_b / (med(t_draft) * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "roofline_verify": {"bound": "hbm", "achieved": verify_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": verify_gbs / peaks["hbm_gbs"], "traffic": traffic.get("verify_kernel"),
+                            "frac": verify_gbs / peaks["hbm_gbs"],
+                            "traffic": traffic.get("verify_kernel") if variant == "a" else None,
                             "algorithmic_bytes": vbytes, "frac_nominal": verify_gbs / NOMINAL_HBM_GBS},
         "roofline_round": {"bound": "hbm", "achieved": round_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                            "frac": round_gbs / peaks["hbm_gbs"], "frac_nominal": round_gbs / NOMINAL_HBM_GBS,
@@ -383,6 +401,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--variant", default="auto", choices=["auto", "a", "b"],
+                    help="a: the draft stores z; b: verify recomputes the rejected rows; auto: b from B = 128 on")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -289,12 +289,6 @@ __device__ __noinline__ int draw_full_row_b(const TcParams& p, int b, int i, dou
   return last_ux * kUnit + max(last, 0);
 }
 
-// Draw request b's token at position i (one warp) by a three-level
-// inverse-CDF search over fp64 sums of the weights exp(z): the G slice sums
-// (whose total is the W that u scales), the chosen slice's sums over its 32-row
-// units, then the chosen unit's 32 weights (from the stored fp32 z, or in
-// variant B from z recomputed for that unit). Writes draft_tokens, q_tok and
-// lse_q; returns the token.
 // Variant B: z of row 32 ux + lane for request b at position i, from the
 // unit's Bf columns staged in shared memory (`sel`: r x 32 bf16, then the
 // operand row) and the position's operand row: base + sum_k a_k Bf[k, v].
@@ -312,9 +306,63 @@ __device__ __forceinline__ float unit_z_staged(const TcParams& p, int b, int i, 
   return __fadd_rn(zb, acc);
 }
 
-template <bool kStoreZ>
-__device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane, const double* t16,
-                                        uint8_t* sel) {
+// Draw request b's token at position i (one warp) by a three-level
+// inverse-CDF search over fp64 sums of the weights exp(z): the G slice sums
+// (whose total is the W that u scales), the chosen slice's sums over its 32-row
+// units, then the chosen unit's 32 weights (from the stored fp32 z). Writes
+// draft_tokens, q_tok and lse_q; returns the token.
+// Inlined into the kernel: as a called function it measured 13% slower (the
+// call kept more of the kernel's registers spilled).
+__device__ __forceinline__ int select_warp(const TcParams& p, int b, int i, int G, int lane, const double* t16) {
+  const DraftArgs& d = p.d;
+  const long long o = static_cast<long long>(b) * d.K + i;
+  const float* zrow = d.z + o * d.V;
+  const double u = static_cast<double>(d.u[o]);
+  const double* part = d.part_S + static_cast<long long>(b) * G;
+  double ex, W;
+  // level 1: slice sums; their total is the W that u scales
+  const int c = warp_search<8>(
+      G, [&](int cc) { return __ldcg(part + cc); },
+      [&](double tot) { return (tot >= kSumLo && tot <= kSumHi) ? u * tot : INFINITY; }, lane, &ex, &W);
+  int tok;
+  double w_t;
+  float shift = 0.f;
+  if (W >= kSumLo && W <= kSumHi) {
+    const double R = u * W - ex;
+    // level 2: the slice's unit sums, in vocabulary order
+    int lo, hi;
+    chunk_bounds(d.V, kUnit, G, c, &lo, &hi);
+    const int ulo = lo / kUnit;
+    const double* us = p.unit_sum + static_cast<long long>(ulo) * d.B + b;
+    double ex2, tot2;
+    const int ux = ulo + warp_search<2>(
+                             (hi - lo) / kUnit, [&](int k) { return __ldcg(us + static_cast<long long>(k) * d.B); },
+                             [&](double) { return R; }, lane, &ex2, &tot2);
+    const double R2 = R - ex2;
+    // level 3: the unit's weights, one per lane
+    const double w = exp_fine(__ldcg(zrow + static_cast<long long>(ux) * kUnit + lane), 0.f, t16);
+    const double inc = warp_inclusive_scan(w);
+    const unsigned hit = __ballot_sync(0xffffffffu, inc > R2 && w > 0.0);
+    const unsigned pos = __ballot_sync(0xffffffffu, w > 0.0);
+    // rounding: the last positive weight of the unit
+    const int x = hit ? __ffs(hit) - 1 : (pos ? 31 - __clz(pos) : 0);
+    w_t = __shfl_sync(0xffffffffu, w, x);
+    tok = ux * kUnit + x;
+  } else {
+    tok = draw_full_row(zrow, d.V, u, lane, b, d.err, &w_t, &shift, &W);
+  }
+  if (lane == 0) {
+    d.tokens[o] = tok;
+    d.q_tok[o] = static_cast<float>(w_t / W);
+    d.lse_q[o] = static_cast<double>(shift) + log(W);
+  }
+  return tok;
+}
+
+// Variant B's draw: select_warp with the last level's 32 logits recomputed
+// from the staged unit (`sel`) instead of read from z.
+__device__ __forceinline__ int select_warp_b(const TcParams& p, int b, int i, int G, int lane, const double* t16,
+                                          uint8_t* sel) {
   const DraftArgs& d = p.d;
   const long long o = static_cast<long long>(b) * d.K + i;
   const double u = static_cast<double>(d.u[o]);
@@ -340,8 +388,7 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
                              [&](double) { return R; }, lane, &ex2, &tot2);
     const double R2 = R - ex2;
     // level 3: the unit's weights, one per lane
-    const float zu = kStoreZ ? __ldcg(d.z + o * d.V + static_cast<long long>(ux) * kUnit + lane)
-                             : unit_z_staged(p, b, i, ux, lane, sel);
+    const float zu = unit_z_staged(p, b, i, ux, lane, sel);
     const double w = exp_fine(zu, 0.f, t16);
     const double inc = warp_inclusive_scan(w);
     const unsigned hit = __ballot_sync(0xffffffffu, inc > R2 && w > 0.0);
@@ -350,8 +397,6 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
     const int x = hit ? __ffs(hit) - 1 : (pos ? 31 - __clz(pos) : 0);
     w_t = __shfl_sync(0xffffffffu, w, x);
     tok = ux * kUnit + x;
-  } else if (kStoreZ) {
-    tok = draw_full_row(d.z + o * d.V, d.V, u, lane, b, d.err, &w_t, &shift, &W);
   } else {
     tok = draw_full_row_b(p, b, i, u, lane, &w_t, &shift, &W);
   }
@@ -366,6 +411,7 @@ __device__ __noinline__ int select_warp(const TcParams& p, int b, int i, int G, 
 // A row of the MMA's B operand for request b at position pos: A[t, :] into
 // the operand image of b's group, K-major with the 128-byte swizzle, and in
 // variant B also into op_rows (one warp).
+template <bool kOpRows>
 __device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t, int pos, int lane) {
   const int gr = b / p.gsize, n = b - gr * p.gsize;
   const int N = round16(group_real(p, gr));
@@ -376,8 +422,7 @@ __device__ __forceinline__ void write_image_row(const TcParams& p, int b, int t,
     const uint4 v = __ldg(A4 + ch);
     const int kb = ch >> 3, c = ch & 7;
     *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) = v;
-    if (p.op_rows != nullptr)
-      reinterpret_cast<uint4*>(p.op_rows + (static_cast<long long>(b) * p.d.K + pos) * p.d.r)[ch] = v;
+    if (kOpRows) reinterpret_cast<uint4*>(p.op_rows + (static_cast<long long>(b) * p.d.K + pos) * p.d.r)[ch] = v;
   }
 }
 
@@ -449,6 +494,7 @@ __device__ __noinline__ void rnn_matvec(const TcParams& p, int b, int lane) {
 // h = tanh(A[t] + U) (U = W h_prev, or 0 at the first position) for request
 // b: stored as the new state and written, rounded to bf16, as b's operand row
 // of position pos (and in variant B into op_rows).
+template <bool kOpRows>
 __device__ __noinline__ void rnn_step(const TcParams& p, int b, int t, bool first, int pos, int lane) {
   const int r = p.d.r, nch = r / 8;
   if (lane >= nch) return;
@@ -472,8 +518,7 @@ __device__ __noinline__ void rnn_step(const TcParams& p, int b, int t, bool firs
   const int kb = lane >> 3, c = lane & 7;
   const uint4 row = make_uint4(out[0], out[1], out[2], out[3]);
   *reinterpret_cast<uint4*>(img + kb * (N * 128) + n * 128 + ((c ^ (n & 7)) << 4)) = row;
-  if (p.op_rows != nullptr)
-    reinterpret_cast<uint4*>(p.op_rows + (static_cast<long long>(b) * p.d.K + pos) * p.d.r)[lane] = row;
+  if (kOpRows) reinterpret_cast<uint4*>(p.op_rows + (static_cast<long long>(b) * p.d.K + pos) * p.d.r)[lane] = row;
 }
 
 // One warp: every lane waits for *ctr >= target (bounded), so the warp stays
@@ -489,12 +534,12 @@ __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned 
 // 19 warps: five share a 16K-register SM sub-partition, so at most 96 registers each
 template <bool kRnn, bool kStoreZ>
 __global__ void __maxnreg__(96)
-    draft_tc_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_bf,
+    draft_tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tm_bf,
                     const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_z) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const DraftArgs& d = p.d;
-  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, p.ngroups * 4 * p.gsize * 8, p.sel_bytes);
+  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, p.ngroups * 4 * p.gsize * 8, kStoreZ ? 0 : p.sel_bytes);
   Bars bars = carve_bars(smem + Ly.bar);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
@@ -661,8 +706,8 @@ __global__ void __maxnreg__(96)
     bool ok = true;
     // position 0's operand: the anchors' rows, and zeros in padded rows
     for (int b = g; b < d.B; b += G) {
-      if (kRnn) rnn_step(p, b, previous_token(d, b, 0), true, 0, lane);
-      else write_image_row(p, b, previous_token(d, b, 0), 0, lane);
+      if (kRnn) rnn_step<!kStoreZ>(p, b, previous_token(d, b, 0), true, 0, lane);
+      else write_image_row<!kStoreZ>(p, b, previous_token(d, b, 0), 0, lane);
     }
     if (g == 0) {
       for (int gr = 0; gr < p.ngroups; ++gr) {
@@ -721,10 +766,11 @@ __global__ void __maxnreg__(96)
           ok = warp_wait_counter(&p.sync_part[slot], static_cast<unsigned>(G), d.err, 0x600u + slot, s_abort, lane);
           if (!ok) break;
           for (int b = first; b < gbase + nreal; b += G) {
-            const int t = select_warp<kStoreZ>(p, b, i, G, lane, t16, smem + Ly.sel);
+            const int t = kStoreZ ? select_warp(p, b, i, G, lane, t16)
+                                  : select_warp_b(p, b, i, G, lane, t16, smem + Ly.sel);
             if (i + 1 < d.K) {
-              if (kRnn) rnn_step(p, b, t, false, i + 1, lane);
-              else write_image_row(p, b, t, i + 1, lane);
+              if (kRnn) rnn_step<!kStoreZ>(p, b, t, false, i + 1, lane);
+              else write_image_row<!kStoreZ>(p, b, t, i + 1, lane);
             }
             ++mine;
           }

@@ -408,6 +408,9 @@ __device__ bool grid_barrier(const Params& P, int k, int* s_flag) {
   return *s_flag != 0;
 }
 
+// kRecompute: variant B (P.recompute), as a template so that variant A's
+// kernel carries none of its code
+template <bool kRecompute>
 __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) uint8_t smem[];
   float* stages = reinterpret_cast<float*>(smem);
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
         mbar_arrive_expect_tx(full, bytes);
         // variant B: evict-first, so that the draft's Bf (evict-last) stays in
         // L2 for the residual kernel that follows
-        if (P.recompute) bulk_load_hint(dst, a.target + ri.row * a.V + v0, bytes, full, policy_evict_first());
+        if (kRecompute) bulk_load_hint(dst, a.target + ri.row * a.V + v0, bytes, full, policy_evict_first());
         else bulk_load(dst, a.target + ri.row * a.V + v0, bytes, full);
       },
       [&](const Desc& ds, const float* stage, uint64_t* empty, int w) { consume_row(P, ds, stage, empty, w, lane); });
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
   if (warp > kProdWarp && n_rows > 0) {
     int r = 0;
     if (warp == kProdWarp + 1) r = sample_p(P, 0, 0.5f, lane, true);
-    if (warp == kProdWarp + 2 && !P.recompute) {
+    if (warp == kProdWarp + 2 && !kRecompute) {
       ResDec d{};
       d.row = P.w.rowinfo[0].row;
       r = residual_token(P, 0, d, 0.5f, lane, true);
@@ -539,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
 
   // variant B: the bonus draws, one warp per request; the residual kernel
   // that follows does the rest
-  if (P.recompute) {
+  if (kRecompute) {
     if (ok) {
       const int n_bonus = static_cast<int>(__ldcg(P.w.ctl + kCtlBonus));
       for (int e = gw; e < n_bonus; e += NW) {
@@ -676,7 +679,8 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
   const size_t smem = static_cast<size_t>(kStages) * kStageBytes + sizeof(Smem);
-  e = cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  auto kernel = P.recompute ? verify_kernel<true> : verify_kernel<false>;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   {
     cudaLaunchAttribute pattr[1];
@@ -712,11 +716,11 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, verify_kernel, P);
+  e = cudaLaunchKernelEx(&cfg, kernel, P);
   if (e == cudaErrorNotSupported) {  // without the early start
     (void)cudaGetLastError();
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, verify_kernel, P);
+    e = cudaLaunchKernelEx(&cfg, kernel, P);
   }
   if (e != cudaSuccess || !P.recompute) return e;
   return launch_residual_tc(P, stream);

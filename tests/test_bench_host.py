@@ -24,6 +24,27 @@ def test_verify_bytes_counts_rows_and_rejected_z_rows():
     assert bench.verify_bytes(151936, 8, np.full(64, 8), np.full(64, 8)) / 1e6 == pytest.approx(350.1, abs=0.05)
 
 
+def test_variant_b_bytes():
+    # variant B: no z write (the operand rows instead); base + Bf is 389.0 MB at qwen3
+    B, K, V, r = 64, 8, 151936, 256
+    got = bench.draft_bytes(B, K, V, r, 2, "b")
+    assert got == B * K * V * 4 + B * K * r * 2 + r * V * 2 + B * K * r * 2 + B * K * (4 + 4 + 8 + 4)
+    assert (got - B * K * r * 4 - B * K * 20) / 1e6 == pytest.approx(389.0, abs=0.05)
+    # verify B reads each rejected request's base row instead of its z row, plus Bf once and the operand rows
+    V, K = 1000, 4
+    L = np.array([4, 0, 2])
+    acc = np.array([4, 0, 1])
+    assert bench.verify_bytes(V, K, L, acc, 64, 2, "b") == (5 + 1 + 3) * V * 4 + V * 4 + 64 * V * 2 + 64 * 2
+    # nothing rejected: no recompute
+    assert bench.verify_bytes(V, K, L, L, 64, 2, "b") == (5 + 1 + 3) * V * 4
+
+
+def test_round_variant_choice():
+    assert bench.round_variant("auto", 64) == "a"
+    assert bench.round_variant("auto", 256) == "b"
+    assert bench.round_variant("a", 512) == "a" and bench.round_variant("b", 1) == "b"
+
+
 def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     (tmp_path / "profiles").mkdir()
