@@ -39,7 +39,7 @@ __device__ __forceinline__ float factor_at(const void* p, long long idx) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(DT, 1) draft_generic_kernel(DraftArgs a) {
+__global__ void __launch_bounds__(DT, 1) draft_generic_kernel(const __grid_constant__ DraftArgs a) {
   extern __shared__ float arow[];  // [RB][r]
   __shared__ double redd[33];
   __shared__ int s_flag;

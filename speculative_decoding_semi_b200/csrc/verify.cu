@@ -12,7 +12,7 @@
 //   plan    one CTA: checks verify_len and the drafted tokens, numbers the
 //           target rows 0..L_b of every request consecutively in request
 //           order and clears the counters of the main kernel.
-//   main    one persistent cooperative CTA per SM, in five phases separated
+//   main    one persistent cooperative CTA per SM, in four phases separated
 //           by device-wide barriers:
 //     1 rows      the target rows stream through a ring of shared-memory
 //                 stages filled by bulk asynchronous copies (one producer
@@ -20,13 +20,16 @@
 //                 stages, reduce 1024-wide segments: fp64 sum of exp(x) and the
 //                 logit at the drafted token;
 //     2 row stats one warp per row: (max, sum) from the segment partials and
-//                 the accept test u * q(t) < p(t) of the row's draft;
-//     3 decide    one warp per request: the first rejection; the request
-//                 joins the list of bonus draws (none) or of residual passes;
-//     4 residual  the rejected rows and their z rows stream through the same
+//                 the accept test u * q(t) < p(t) of the row's draft; the warp
+//                 that completes a request's last row (a per-request counter)
+//                 finds its first rejection, and the request joins the list
+//                 of bonus draws (none) or of residual passes;
+//     3 residual  the rejected rows and their z rows stream through the same
 //                 ring: sums of max(0, p - q) over 512-wide segments; the
 //                 warps outside the stream make the bonus draws meanwhile;
-//     5 resample  one warp per listed request draws the resampled token.
+//     4 resample  one warp per listed request draws the resampled token.
+// (Variant B ends after phase 2 with the bonus draws: its residual kernel
+// recomputes the rejected rows of z and draws the rest.)
 // The barriers fall between streaming phases, when no copy is in flight: a
 // gpu-scope fence on an SM with bulk copies in flight waits for them to land,
 // and a plain store from such an SM takes several microseconds to be seen by
@@ -108,6 +111,7 @@ __global__ void __launch_bounds__(kPlanThreads) verify_plan_kernel(Params p) {
     if (b < a.B) {
       const int r0 = carry + ex;
       p.w.rowbase[b] = valid ? r0 : -1;
+      p.w.req_rows[b] = 0u;
       if (valid) {
         for (int rho = 0; rho <= L; ++rho) {
           int tok = -1;
@@ -182,10 +186,10 @@ __device__ void row_stats(const Params& P, int R, int lane) {
   }
 }
 
-// Phase 3, one warp: request b's first rejection; a place in the list of
+// Phase 2, one warp: request b's first rejection; a place in the list of
 // bonus draws, or the residual pass's inputs and a place in its list.
 // With `warm` set it writes nothing: it runs once during phase 1 to load its
-// code into the SM's instruction cache ahead of phase 3.
+// code into the SM's instruction cache ahead of phase 2.
 __device__ __noinline__ void decide(const Params& P, int b, int lane, bool warm = false) {
   const VerifyArgs& a = P.a;
   const int r0 = P.w.rowbase[b];
@@ -261,7 +265,7 @@ __device__ __noinline__ void decide(const Params& P, int b, int lane, bool warm 
   }
 }
 
-// Phase 5, one warp: the resampled token of listed request b.
+// Phase 4, one warp: the resampled token of listed request b.
 // The resampled token of request b from its residual segment sums; `warm`
 // as for sample_p.
 __device__ __noinline__ int residual_token(const Params& P, int b, const ResDec& d, float u, int lane, bool warm) {
@@ -530,14 +534,22 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
   }
   ok = __syncthreads_and(ok) && grid_barrier(P, 0, &s_flag);
 
-  // ---- phase 2: row statistics and accept tests
+  // ---- phase 2: row statistics and accept tests; the warp that completes
+  // the last row of a request makes its decision (the bonus and residual
+  // lists), so no device-wide barrier separates the two
   if (ok)
-    for (int R = gw; R < n_rows; R += NW) row_stats(P, R, lane);
-  ok = ok && grid_barrier(P, 1, &s_flag);
-
-  // ---- phase 3: decisions; the bonus and residual lists
-  if (ok)
-    for (int b = gw; b < a.B; b += NW) decide(P, b, lane);
+    for (int R = gw; R < n_rows; R += NW) {
+      row_stats(P, R, lane);
+      const int brl = P.w.rowinfo[R].brl;
+      const int b = brl & 0xffff, L = brl >> 22;
+      unsigned done = 0;
+      if (lane == 0) done = atom_add_acq_rel_gpu(P.w.req_rows + b, 1u);  // releases this row's results
+      if (__shfl_sync(0xffffffffu, done, 0) == static_cast<unsigned>(L)) {
+        // every lane acquires the request's other rows before reading them
+        (void)ld_acquire_gpu(P.w.req_rows + b);
+        decide(P, b, lane);
+      }
+    }
   ok = ok && grid_barrier(P, 2, &s_flag);
 
   // variant B: the bonus draws, one warp per request; the residual kernel
@@ -552,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
       }
     }
   } else {
-    // ---- phase 4: residual segment sums of the listed requests
+    // ---- phase 3: residual segment sums of the listed requests
     const int n_listed = ok ? static_cast<int>(__ldcg(P.w.ctl + kCtlListed)) : 0;
     if (ok) {
       const uint64_t pol_first = policy_evict_first();
@@ -600,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
       ok = __syncthreads_and(ok) && grid_barrier(P, 3, &s_flag);
     }
 
-    // ---- phase 5: resampled tokens
+    // ---- phase 4: resampled tokens
     if (ok)
       for (int e = gw; e < n_listed; e += NW) resample(P, __ldcg(P.w.list + e), lane);
   }
@@ -613,7 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1) verify_kernel(const __grid_consta
 }
 
 struct Layout {
-  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, blist, seg_w, slots, total;
+  size_t rowinfo, rowbase, ctl, part_m, part_S, x_tok, rstat, accepted, dec, resfac, list, blist, seg_w, slots, req_rows,
+      total;
 };
 
 Layout verify_layout(int B, int K, int V) {
@@ -640,6 +653,7 @@ Layout verify_layout(int B, int K, int V) {
   L.blist = take(nb * sizeof(int));
   L.seg_w = take(nb * nrseg * sizeof(double));
   L.slots = take(nb * sizeof(ResSlot));
+  L.req_rows = take(nb * sizeof(unsigned));
   L.total = off;
   return L;
 }
@@ -670,6 +684,7 @@ cudaError_t launch_verify(VerifyArgs a, char* region, cudaStream_t stream) {
   P.w.blist = reinterpret_cast<int*>(region + L.blist);
   P.w.seg_w = reinterpret_cast<double*>(region + L.seg_w);
   P.w.slots = reinterpret_cast<ResSlot*>(region + L.slots);
+  P.w.req_rows = reinterpret_cast<unsigned*>(region + L.req_rows);
   P.recompute = a.z == nullptr ? 1 : 0;
   P.res_gsize = residual_group_size(a.B);
 

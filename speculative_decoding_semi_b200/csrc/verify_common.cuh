@@ -84,6 +84,7 @@ struct Ws {
   float2* resfac;    // [B][nseg] residual (shift, p factor) per 1024-segment
   int* list;         // [B] requests with a residual pass
   int* blist;        // [B] requests whose drafts were all accepted (bonus draw)
+  unsigned* req_rows;  // [B] rows of the request whose statistics are done (phase 2)
   double* seg_w;     // [B][nrseg] residual segment sums
   ResSlot* slots;    // [B] variant B: the requests with a residual, in list order
 };
