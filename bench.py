@@ -257,8 +257,8 @@ def run_gpu(args):
     bufs = rnd.RoundBuffers(B, K, V, r, variant=variant)
     stream = torch.cuda.Stream()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-    # draft, schedule (rank, final), verify (plan, main), and variant B's residual kernel
-    launches_per_round = 1 + 2 + 2 + (1 if variant == "b" else 0)
+    # draft, schedule, verify (plan, main), and variant B's residual kernel
+    launches_per_round = 1 + 1 + 2 + (1 if variant == "b" else 0)
 
     def one_round(ev=None):
         with torch.cuda.stream(stream):

@@ -55,7 +55,9 @@ typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype;
  * workspace serves a whole round). Returns 0 if the sizes are out of range. */
 size_t dspark_workspace_bytes(int B, int K, int V, int r);
 
-/* Zero `ws_bytes` bytes of a fresh workspace on `stream` (clears the error word). */
+/* Zero `ws_bytes` bytes of a fresh workspace on `stream` (clears the error word
+ * and the device-wide counters the kernels keep in it; a workspace must be
+ * initialised once before its first use). */
 dspark_status dspark_workspace_init(void* workspace, size_t ws_bytes, dspark_stream_t stream);
 
 /*
@@ -250,9 +252,10 @@ dspark_status dspark_advance_anchor(const int32_t* out_tokens, const int32_t* n_
  * current device (cudaGetSymbolAddress, which allocates nothing); the first
  * call on a device may load the library's device code, so make it before any
  * stream capture. All calls share the one
- * array, and each call fully rewrites what it reads back, so no state carries
- * over between calls; calls that overlap on the GPU (two streams, or two
- * threads) race on the array and must be serialised by the caller.
+ * array, and each call fully rewrites what it reads back (its one counter
+ * returns to zero at the end of the call), so no state carries over between
+ * calls; calls that overlap on the GPU (two streams, or two threads) race on
+ * the array and must be serialised by the caller.
  */
 #define DSPARK_STATIC_SCHEDULE_MAX_ITEMS 16384
 dspark_status dspark_schedule_static(const float* conf_logits, const float* temps,

@@ -67,6 +67,7 @@ struct ScheduleArgs {
   unsigned* err;
   int32_t* rank;        // [B*K]
   double* sorted_P;     // [B*K]
+  unsigned* done;       // CTAs finished (the last one runs the final step); zero between calls
 };
 
 size_t draft_scratch_bytes(int B, int K, int V, int r);

@@ -20,11 +20,15 @@ pytestmark = pytest.mark.gpu
 
 
 def test_tiny_many_seeds():
+    """The survey's volume for the tiny workload: 10,000 seeds (one set of
+    buffers and one workspace for all of them)."""
+    from speculative_decoding_semi_b200 import round as rnd
     t = parity.Tally()
-    for seed in range(2000):
+    bufs = rnd.RoundBuffers(4, 4, 1024, 32)
+    for seed in range(10000):
         inp = synth.make_round(0, seed=5000 + seed)
-        parity.check_round(inp, tally=t)
-    t.check("tiny x2000")
+        parity.check_round(inp, tally=t, bufs=bufs)
+    t.check("tiny x10000")
 
 
 @pytest.mark.parametrize("like,sizes", [

@@ -87,6 +87,21 @@ def test_variant_b_full_size(key, sample):
     t.check(f"variant b {key}")
 
 
+@pytest.mark.parametrize("key,seeds,sample", [("qwen3", 6, 8), ("latency", 40, None), ("highconc", 2, 16),
+                                             ("mixed", 2, 16)])
+def test_variant_b_seed_volume(key, seeds, sample):
+    """More seeds of every full-size workload in variant B, the excused
+    near-ties pooled; the Markov factors drawn once per workload."""
+    t = parity.Tally()
+    factors = synth.make_factors(key)
+    for k in range(seeds):
+        inp = synth.make_round(key, seed=7500 + k, factors=factors)
+        B = inp["base"].shape[0]
+        reqs = None if sample is None else np.unique(np.linspace(k % 3, B - 1, sample).astype(int))
+        parity.check_round(inp, requests=reqs, tally=t, variant="b")
+    t.check(f"variant b {key} x{seeds}")
+
+
 def test_variant_b_agrees_with_variant_a():
     """Same inputs, both variants: the drafts are the same computation (z from
     the same tensor-core GEMM) and the verify outputs follow the definition, so
