@@ -143,7 +143,8 @@ __device__ void final_step(const ScheduleArgs& a) {
 
 template <int ST>
 __global__ void __launch_bounds__(ST) schedule_kernel(ScheduleArgs a, int tpi) {
-  extern __shared__ double P[];  // [B*K]
+  extern __shared__ double Pt[];  // [K][B]: position-major, so that lanes searching consecutive requests read
+                                  // consecutive words
   __shared__ int s_last;
   // launched early (programmatic dependent launch): the previous kernel's
   // writes are visible after the wait; the next kernel may launch meanwhile
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(ST) schedule_kernel(ScheduleArgs a, int tpi) {
       const double x = static_cast<double>(a.conf[b * K + j]) / static_cast<double>(a.temps[j]);
       const double s = 1.0 / (1.0 + exp(-x));
       prod = __dmul_rn(prod, s);
-      P[b * K + j] = prod;
+      Pt[j * B + b] = prod;
       if (blockIdx.x == 0) a.survival[b * K + j] = static_cast<float>(prod);
     }
   }
@@ -170,14 +171,14 @@ __global__ void __launch_bounds__(ST) schedule_kernel(ScheduleArgs a, int tpi) {
     const int item = base + threadIdx.x / tpi;
     const bool valid = item < N;
     const int b = valid ? item / K : 0, j = valid ? item - b * K : 0;
-    const double p = valid ? P[item] : 0.0;
+    const double p = valid ? Pt[j * B + b] : 0.0;
     int cnt = 0;
     if (valid) {
       for (int bp = lane; bp < B; bp += tpi) {
         int lo = 0, hi = K;
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
-          if (precedes(P[bp * K + mid], mid, bp, p, j, b)) lo = mid + 1;
+          if (precedes(Pt[mid * B + bp], mid, bp, p, j, b)) lo = mid + 1;
           else hi = mid;
         }
         cnt += lo;
