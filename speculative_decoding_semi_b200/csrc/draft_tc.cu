@@ -81,6 +81,7 @@ constexpr int kMaxAccSlots = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarBytes = 2048;
 constexpr int kSubPerWarp = kMaxGroup / kSub / 4;  // sub-chunks of a group per epilogue warp
+static_assert(kSubPerWarp == 2, "the spread mode's running totals assume two sub-chunks per warp");
 constexpr double kSumLo = 1e-280, kSumHi = 1e280;  // row sums handled with the fixed shift
 
 
@@ -102,6 +103,7 @@ struct TcParams {
   double* ustate;       // [B][r] RNN head: W h_i, formed while position i streams
   uint16_t* op_rows;    // [B][K][r] variant B: the operand row of every position (bf16), or null
   int sel_bytes;        // variant B: shared staging of the last search level (0 in variant A)
+  int spread;           // B <= 32: the kernel's kSpread instance (a quadrant's warps take turns over the tiles)
 };
 
 struct Layout {
@@ -154,6 +156,26 @@ __device__ __forceinline__ int chunks_for(int ncol, int hh) {
   return nsub > hh ? (nsub - hh + 3) / 4 : 0;
 }
 
+// The sub-chunks (16 requests each) that epilogue warp h of a quadrant takes
+// in the t-th tile it visits in group gr: normally those with index
+// s = 4k + (h + gr) % 4, in every tile (item_count of them). With at most two
+// sub-chunks (kSpread, B <= 32) most warps would have none; there the items
+// (t, s) are dealt round-robin over the quadrant's four warps instead, item
+// t * nsub + s to warp (t * nsub + s) % 4, so each warp takes at most one
+// per tile.
+__device__ __forceinline__ int spread_sub(int h, int t, int nsub) { return ((h - t * nsub) % 4 + 4) % 4; }
+template <bool kSpread>
+__device__ __forceinline__ int item_count(const TcParams& p, int gr, int h, int t) {
+  const int nreal = group_real(p, gr);
+  if (!kSpread) return chunks_for(nreal, half_of(h, gr));
+  return spread_sub(h, t, (nreal + kSub - 1) / kSub) < (nreal + kSub - 1) / kSub ? 1 : 0;
+}
+template <bool kSpread>
+__device__ __forceinline__ int item_sub(const TcParams& p, int gr, int h, int t, int k) {
+  if (!kSpread) return 4 * k + half_of(h, gr);
+  return spread_sub(h, t, (group_real(p, gr) + kSub - 1) / kSub);
+}
+
 // Tile visited t-th in pass (i, gr): passes over the slice alternate
 // direction, so each pass starts on the Bf tiles the previous one touched last
 // (the ones most likely still in L2).
@@ -164,6 +186,7 @@ __device__ __forceinline__ int phys_tile(int i, int gr, int ngroups, int ntiles,
 // The sequence of (position, group, tile, chunk) boxes one epilogue warp
 // streams, in consumption order; the TMA refill cursor walks it ahead of the
 // consumer across positions.
+template <bool kSpread>
 struct Items {
   const TcParams* p;
   int ntiles, last_rows, q, h;
@@ -187,7 +210,7 @@ struct Items {
         ++gr;
         continue;
       }
-      if (!tile_ok() || k >= chunks_for(group_real(*p, gr), half_of(h, gr))) {
+      if (!tile_ok() || k >= item_count<kSpread>(*p, gr, h, t)) {
         k = 0;
         ++t;
         continue;
@@ -532,14 +555,15 @@ __device__ __forceinline__ bool warp_wait_counter(const unsigned* ctr, unsigned 
 }
 
 // 19 warps: five share a 16K-register SM sub-partition, so at most 96 registers each
-template <bool kRnn, bool kStoreZ>
+template <bool kRnn, bool kStoreZ, bool kSpread>
 __global__ void __maxnreg__(96)
     draft_tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ CUtensorMap tm_bf,
                     const __grid_constant__ CUtensorMap tm_base, const __grid_constant__ CUtensorMap tm_z) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const DraftArgs& d = p.d;
-  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, p.ngroups * 4 * p.gsize * 8, kStoreZ ? 0 : p.sel_bytes);
+  const Layout Ly = make_layout(p.nbf, p.image_stride, p.nbs, (kSpread ? kEpiWarps : p.ngroups * 4) * p.gsize * 8,
+                                kStoreZ ? 0 : p.sel_bytes);
   Bars bars = carve_bars(smem + Ly.bar);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
@@ -746,10 +770,13 @@ __global__ void __maxnreg__(96)
           ok = false;
           break;
         }
-        // this CTA's slice sums, summed over the four quadrants in a fixed order
+        // this CTA's slice sums, summed over the four quadrants (spread: the
+        // sixteen epilogue warps) in a fixed order
         const double* sp = s_part + gr * 4 * p.gsize;
         for (int n = lane; n < nreal; n += 32) {
-          const double S = sp[n] + sp[p.gsize + n] + sp[2 * p.gsize + n] + sp[3 * p.gsize + n];
+          double S = sp[n] + sp[p.gsize + n] + sp[2 * p.gsize + n] + sp[3 * p.gsize + n];
+          if (kSpread)
+            for (int w = 4; w < kEpiWarps; ++w) S += sp[w * p.gsize + n];
           d.part_S[static_cast<long long>(gbase + n) * G + g] = S;
           d.part_m[static_cast<long long>(gbase + n) * G + g] = 0.f;
         }
@@ -796,7 +823,7 @@ __global__ void __maxnreg__(96)
     }
     float* ring = reinterpret_cast<float*>(smem + Ly.ring + warp * p.nbs * kBoxBytes);
     uint64_t* rfull = bars.base_full(warp * kMaxRingSlots);
-    Items L;
+    Items<kSpread> L;
     L.p = &p;
     L.ntiles = ntiles;
     L.last_rows = last_rows;
@@ -808,7 +835,7 @@ __global__ void __maxnreg__(96)
       const int j = nl % p.nbs;
       mbar_arrive_expect_tx(&rfull[j], kBoxBytes);
       tma_load_3d(ring + j * (kBoxBytes / 4), &tm_base, lo + L.ptile() * kTileRows + kUnit * q, L.i,
-                  L.gr * p.gsize + (4 * L.k + half_of(h, L.gr)) * kSub, &rfull[j], pol_first);
+                  L.gr * p.gsize + item_sub<kSpread>(p, L.gr, h, L.t, L.k) * kSub, &rfull[j], pol_first);
       L.next();
       ++nl;
     };
@@ -847,7 +874,8 @@ __global__ void __maxnreg__(96)
         const int gbase = gr * p.gsize;
         const int nreal = group_real(p, gr);
         const int hh = half_of(h, gr);
-        const int nk = chunks_for(nreal, hh);
+        const int nk = kSpread ? 1 : chunks_for(nreal, hh);
+        const int nsub = (nreal + kSub - 1) / kSub;
         // lane 2c sums column (request) col0 + c of each sub-chunk over the slice
         double acc[kSubPerWarp];
 #pragma unroll
@@ -862,14 +890,16 @@ __global__ void __maxnreg__(96)
           tc_fence_after();
           if (kUnit * q < rows) {
             const int v0 = lo + pt * kTileRows + kUnit * q;
+            const int nkt = kSpread ? item_count<kSpread>(p, gr, h, t) : nk;
+            const int ssub = kSpread ? spread_sub(h, t, nsub) : 0;
 #pragma unroll
             for (int kk = 0; kk < kSubPerWarp; ++kk) {
-              if (kk < nk && ok) {
+              if (kk < nkt && ok) {
                 const int j = nc % p.nbs;
                 ok = mbar_wait(&rfull[j], (nc / p.nbs) & 1, s_abort, d.err, 0x301u);
                 if (ok) {
                   float* box = ring + j * (kBoxBytes / 4);
-                  const int col0 = (4 * kk + hh) * kSub;
+                  const int col0 = (kSpread ? ssub : 4 * kk + hh) * kSub;
                   uint32_t rg[kSub];
                   tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(kUnit * q) << 16) +
                                          static_cast<uint32_t>(slot * p.slot_stride + col0),
@@ -903,7 +933,9 @@ __global__ void __maxnreg__(96)
                   const double us = warp_transpose_sum16(wv, lane);
                   const int col = gbase + col0 + cr;
                   if ((lane & 1) == 0 && col0 + cr < nreal) {
-                    acc[kk] += us;
+                    // (spread: the sub-chunk index picks the running total)
+                    if (!kSpread || ssub == kk) acc[kk] += us;
+                    else acc[kSubPerWarp - 1 - kk] += us;
                     p.unit_sum[static_cast<long long>(v0 / kUnit) * d.B + col] = us;
                   }
                   if (lane == 0) {
@@ -924,11 +956,17 @@ __global__ void __maxnreg__(96)
           if (pending >= 0 && nc - mark > 0) release_pending(nc - mark);
         }
         if (!ok) break;
-        // this warp's quadrant of the slice sums of group gr
+        // this warp's quadrant of the slice sums of group gr (spread: this
+        // warp's share of them, one row of partials per warp)
 #pragma unroll
         for (int kk = 0; kk < kSubPerWarp; ++kk) {
-          const int col = (4 * kk + hh) * kSub + (lane >> 1);
-          if ((lane & 1) == 0 && kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[kk];
+          if (kSpread) {
+            const int col = kk * kSub + (lane >> 1);
+            if ((lane & 1) == 0 && kk < nsub && col < nreal) s_part[warp * p.gsize + col] = acc[kk];
+          } else {
+            const int col = (4 * kk + hh) * kSub + (lane >> 1);
+            if ((lane & 1) == 0 && kk < nk && col < nreal) s_part[(gr * 4 + q) * p.gsize + col] = acc[kk];
+          }
         }
         release_pending(0);
         pending = gr;
@@ -1006,7 +1044,8 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
   int dev = 0, max_smem = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int part_bytes = p.ngroups * 4 * p.gsize * 8;
+  p.spread = a.B <= 2 * kSub ? 1 : 0;  // one group of at most two sub-chunks
+  const int part_bytes = (p.spread ? kEpiWarps : p.ngroups * 4) * p.gsize * 8;
   p.sel_bytes = a.z == nullptr ? a.r * kUnit * 2 + a.r * 2 : 0;
   // deepest Bf and base rings that fit, favouring at least 4 base slots
   const int choices[][2] = {{6, 4}, {4, 4}, {6, 3}, {4, 3}, {4, 2}, {3, 2}, {2, 2}};
@@ -1040,11 +1079,15 @@ cudaError_t launch_draft_tc(DraftArgs a, int G, unsigned* sync, char* extra, cud
   // the Markov head's kernel carries no code of the RNN head, and variant A's
   // none of variant B's
   const bool store_z = a.z != nullptr;
-  const void* fn = a.W != nullptr
-                       ? (store_z ? reinterpret_cast<const void*>(&draft_tc_kernel<true, true>)
-                                  : reinterpret_cast<const void*>(&draft_tc_kernel<true, false>))
-                       : (store_z ? reinterpret_cast<const void*>(&draft_tc_kernel<false, true>)
-                                  : reinterpret_cast<const void*>(&draft_tc_kernel<false, false>));
+  // one instance per (head, variant, small batch)
+  using KernelFn = void (*)(const TcParams, const CUtensorMap, const CUtensorMap, const CUtensorMap);
+  static const KernelFn kernels[8] = {
+      draft_tc_kernel<false, false, false>, draft_tc_kernel<false, false, true>,
+      draft_tc_kernel<false, true, false>,  draft_tc_kernel<false, true, true>,
+      draft_tc_kernel<true, false, false>,  draft_tc_kernel<true, false, true>,
+      draft_tc_kernel<true, true, false>,   draft_tc_kernel<true, true, true>};
+  const void* fn = reinterpret_cast<const void*>(
+      kernels[(a.W != nullptr ? 4 : 0) + (store_z ? 2 : 0) + (p.spread ? 1 : 0)]);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   int per_sm = 0;
