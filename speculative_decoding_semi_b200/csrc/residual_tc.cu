@@ -61,7 +61,6 @@ constexpr int kBoxFloats = kSub * kUnit;      // one box of base or of target lo
 constexpr int kSlotBytes = 2 * kBoxFloats * 4;
 constexpr int kMaxGroup = 128;
 constexpr int kMaxGroups = 4;
-constexpr int kMaxRing = 4;
 constexpr int kMaxAccSlots = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSubPerWarp = kMaxGroup / kSub / 2;
@@ -564,7 +563,7 @@ cudaError_t launch_residual_tc(const Params& P, cudaStream_t stream) {
   const VerifyArgs& a = P.a;
   RsParams rp{};
   rp.P = P;
-  rp.gsize = std::min(kMaxGroup, std::max(32, (a.B + 31) & ~31));
+  rp.gsize = P.res_gsize;  // the groups the verify kernel laid the operand images out for
   if ((a.B + rp.gsize - 1) / rp.gsize > kMaxGroups) return cudaErrorInvalidValue;
   rp.r_stages = a.r / kKStage;
   rp.slot_stride = (rp.gsize + 31) & ~31;

@@ -8,7 +8,7 @@
 // number; if every draft passes sample the next token from the target, else
 // resample from an adjusted distribution (here max(0, p - q) renormalised).
 //
-// Two launches.
+// Two launches (variant B adds the residual kernel of residual_tc.cu).
 //   plan    one CTA: checks verify_len and the drafted tokens, numbers the
 //           target rows 0..L_b of every request consecutively in request
 //           order and clears the counters of the main kernel.

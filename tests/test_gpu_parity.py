@@ -20,8 +20,8 @@ pytestmark = pytest.mark.gpu
 
 
 def test_tiny_many_seeds():
-    """The survey's volume for the tiny workload: 10,000 seeds (one set of
-    buffers and one workspace for all of them)."""
+    """10,000 seeds of the tiny workload (one set of buffers and one
+    workspace for all of them)."""
     from speculative_decoding_semi_b200 import round as rnd
     t = parity.Tally()
     bufs = rnd.RoundBuffers(4, 4, 1024, 32)
