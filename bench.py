@@ -77,7 +77,10 @@ class ClockSampler:
                0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period: float = 0.004):
+    # 0.5 ms: a short timed region (20 rounds at qwen3 are ~10 ms on the GPU)
+    # still gets ten or more samples; the sampler is a host thread, and the
+    # rounds are timed by CUDA events, so it does not enter the measurement
+    def __init__(self, index: int, period: float = 0.0005):
         self.samples, self.reasons, self.period = [], set(), period
         self.ok = False
         try:
