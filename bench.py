@@ -124,16 +124,23 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def cpu_baseline(inp: dict, seconds: float = 15.0) -> dict:
-    """The oracle as it stands, on host cores, on a bounded sample of requests."""
-    import oracle
+def cpu_model() -> str:
     try:
-        import threadpoolctl
-        cores = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
-    except Exception:
-        cores = os.cpu_count() or 1
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_rate(inp: dict, seconds: float, n_req: int = 4):
+    """Rounds/s of the oracle from rounds on n_req requests, scaled to the batch."""
+    import oracle
     B = inp["base"].shape[0]
-    n_req, rounds, spent = 4, 0, 0.0
+    rounds, spent = 0, 0.0
     t_start = time.perf_counter()
     while spent < seconds and rounds < 64:
         reqs = (np.arange(n_req) + rounds * n_req) % B
@@ -143,11 +150,32 @@ def cpu_baseline(inp: dict, seconds: float = 15.0) -> dict:
         rounds += 1
         if time.perf_counter() - t_start > 2 * seconds:
             break
-    sec_per_round = spent / rounds * (B / n_req)
-    return {"value": 1.0 / sec_per_round, "unit": "rounds/s", "cores": int(cores), "kind": "oracle",
-            "extrapolated": True,
-            "sample": f"{rounds} oracle rounds of {n_req} of {B} requests each (draft+verify per request, "
-                      f"schedule on the full batch), scaled by {B}/{n_req}; {spent:.1f} s of CPU work"}
+    return 1.0 / (spent / rounds * (B / n_req)), rounds, spent
+
+
+def cpu_baseline(inp: dict, seconds: float = 15.0, single_thread_seconds: float = 0.0) -> dict:
+    """The oracle as it stands, on host cores, on a bounded sample of requests
+    (numpy's own thread pool over the host cores; with single_thread_seconds,
+    also one thread)."""
+    try:
+        import threadpoolctl
+        cores = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
+    except Exception:
+        threadpoolctl = None
+        cores = os.cpu_count() or 1
+    B = inp["base"].shape[0]
+    n_req = 4
+    value, rounds, spent = _oracle_rate(inp, seconds, n_req)
+    out = {"value": value, "unit": "rounds/s", "cores": int(cores), "kind": "oracle",
+           "extrapolated": True, "host_cpus": os.cpu_count(), "cpu_model": cpu_model(),
+           "sample": f"{rounds} oracle rounds of {n_req} of {B} requests each (draft+verify per request, "
+                     f"schedule on the full batch), scaled by {B}/{n_req}; {spent:.1f} s of CPU work"}
+    if single_thread_seconds > 0 and threadpoolctl is not None:
+        with threadpoolctl.threadpool_limits(limits=1):
+            v1, r1, s1 = _oracle_rate(inp, single_thread_seconds, n_req)
+        out["single_thread"] = {"value": v1, "unit": "rounds/s", "cores": 1,
+                                "sample": f"{r1} rounds of {n_req} requests, scaled; {s1:.1f} s"}
+    return out
 
 
 def source_digest() -> str:
@@ -350,7 +378,7 @@ def run_gpu(args):
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(inp, seconds=args.cpu_seconds)
+        cb = cpu_baseline(inp, seconds=args.cpu_seconds, single_thread_seconds=min(5.0, args.cpu_seconds / 3))
 
     traffic = measured_traffic(w.name)
     line = {
@@ -398,7 +426,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="qwen3")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
