@@ -4,7 +4,8 @@ recomputed on the tensor cores) against the CPU oracle.
 The oracle is the same as for variant A: the method's definition does not
 change, only where z lives. Cases: shapes with ragged last tiles and
 vocabulary slices of one quadrant; batches whose rejected requests fill one,
-two and four residual groups (N = 128 per group); the RNN head; packed ragged
+two and four residual groups (N = 128 per group); no rejected request at all;
+one request with one position; the RNN head; packed ragged
 target rows; full-size workloads on sampled requests; extreme logits (p
 weighed with the row's own shift; the slow redraw of a draft row beyond the
 fixed-shift range without stored z); and variant A and B on the same inputs.
@@ -156,6 +157,33 @@ def test_variant_b_rows_beyond_fp64_range():
         toks = g["draft"]["tokens"]
         assert np.all((toks >= 0) & (toks < w.V))
     assert not t.failures, t.failures[:10]
+
+
+def test_variant_b_no_residual():
+    """Nothing to resample: every verify length 0 (a profile that makes any
+    verified token too expensive), and every draft accepted (u_accept = 0);
+    the residual kernel then has no group and only the bonus draws remain."""
+    w = synth.custom(1, B=10, K=4, V=4096, r=64, n_prof=40)
+    inp = synth.make_round(w, seed=3)
+    inp["profile"] = (1.0 + 1000.0 * np.maximum(np.arange(1, 41) - 10, 0)).astype(np.float32)
+    t, g = parity.check_round(inp, variant="b")
+    t.check()
+    assert np.all(g["schedule"]["verify_len"] == 0)
+    assert np.all(g["verify"]["n_out"] == 1)
+    inp = synth.make_round(w, seed=4)
+    inp["u_accept"] = np.zeros_like(inp["u_accept"])
+    t, g = parity.check_round(inp, variant="b")
+    t.check()
+    assert np.all(g["verify"]["accepted"] == g["schedule"]["verify_len"])
+
+
+def test_variant_b_single_request():
+    for V in (64, 151936):
+        w = synth.custom(1, B=1, K=1, V=V, r=64, n_prof=4)
+        t = parity.Tally()
+        for seed in range(3):
+            parity.check_round(synth.make_round(w, seed=seed), tally=t, variant="b")
+        t.check()
 
 
 def test_variant_b_unsupported_shapes():
