@@ -45,6 +45,43 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": HBM_FALLBACK_GBS, "source": "fallback"}
 
 
+def l2_read_gbs(stream, mb: int = 32, passes: int = 64, reps: int = 5):
+    """Read bandwidth from L2 in GB/s: the probe library (libdspark_probe.so)
+    reads an L2-resident buffer of `mb` MB `passes` times with L2-only 16-byte
+    loads; the median of `reps` timed launches on `stream`, after two untimed
+    ones that also make the buffer resident. None when the probe is missing or
+    fails (the bench line then carries no L2 fraction)."""
+    try:
+        import ctypes
+        import torch
+        lib = ctypes.CDLL(os.path.join(ROOT, "speculative_decoding_semi_b200", "libdspark_probe.so"))
+        lib.dspark_probe_sink_words.restype = ctypes.c_size_t
+        lib.dspark_probe_l2_read.restype = ctypes.c_int
+        lib.dspark_probe_l2_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p,
+                                             ctypes.c_size_t, ctypes.c_void_p]
+        words = int(lib.dspark_probe_sink_words())
+        nbytes = mb * 1024 * 1024
+        buf = torch.ones(nbytes // 4, dtype=torch.float32, device="cuda")
+        sink = torch.empty(max(words, 1), dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+        times = []
+        for k in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            st = lib.dspark_probe_l2_read(ctypes.c_void_p(buf.data_ptr()), nbytes, passes,
+                                          ctypes.c_void_p(sink.data_ptr()), words,
+                                          ctypes.c_void_p(stream.cuda_stream))
+            e1.record(stream)
+            if st != 0:
+                return None
+            e1.synchronize()
+            if k >= 2:
+                times.append(e0.elapsed_time(e1))
+        return nbytes * passes / (statistics.median(times) * 1e-3) / 1e9
+    except Exception:
+        return None
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -376,6 +413,19 @@ def run_gpu(args):
                "note": "Markov factors are model weights kept resident; per-round logits, confidences "
                        "and uniforms are copied in, emitted tokens copied out"}
 
+    # the draft reads Bf once per position; with few requests per position
+    # those reads come from L2, so their rate is also set against L2's
+    l2_gbs = l2_read_gbs(stream)
+    bf_reads = K * r * V * fb
+    bf_gbs = bf_reads / (med(t_draft) * 1e-3) / 1e9
+    roofline_l2 = None
+    if l2_gbs:
+        roofline_l2 = {"bound": "l2", "kernel": "dspark_markov_draft" + ("_b" if variant == "b" else ""),
+                       "achieved": bf_gbs, "peak": l2_gbs, "unit": "GB/s", "frac": bf_gbs / l2_gbs,
+                       "bytes": bf_reads,
+                       "note": "Bf [r,V] read at each of the K positions, against the L2 read bandwidth "
+                               "measured in this run (32 MB resident buffer, L2-only 16-byte loads)"}
+
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(inp, seconds=args.cpu_seconds, single_thread_seconds=min(5.0, args.cpu_seconds / 3))
@@ -407,6 +457,7 @@ def run_gpu(args):
         "roofline_round": {"bound": "hbm", "achieved": round_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                            "frac": round_gbs / peaks["hbm_gbs"], "frac_nominal": round_gbs / NOMINAL_HBM_GBS,
                            "algorithmic_bytes": dbytes + vbytes},
+        "roofline_l2": roofline_l2,
         "round_stats": {"verify_tokens": int((L + 1).sum()), "accepted_mean": float(acc.mean()),
                         "emitted_per_round": int(n_out.sum())},
         "gpu_launches": launches_per_round * args.steps,

@@ -4,6 +4,8 @@ Usage: python speculative_decoding_semi_b200/build.py [--verbose] [--ptxas]
 Each .cu under csrc/ is compiled in parallel to an object file under _build/,
 then linked into speculative_decoding_semi_b200/libdspark.so with the CUDA
 runtime linked statically (the library then needs only the driver at run time).
+The L2 read probe under probe/ (not part of the library's path; the benchmark
+loads it for its L2 denominator) becomes libdspark_probe.so the same way.
 """
 from __future__ import annotations
 
@@ -18,6 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libdspark.so")
+PROBE_SRC = os.path.join(HERE, "probe", "l2_read.cu")
+PROBE_LIB = os.path.join(HERE, "libdspark_probe.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -68,6 +72,8 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
                 print(out)
     if jobs or _needs_rebuild(LIB, objs):
         run([nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs])
+    if _needs_rebuild(PROBE_LIB, [PROBE_SRC]):
+        run([nvcc(), *ARCH, *FLAGS, "-shared", "-cudart", "static", "-o", PROBE_LIB, PROBE_SRC])
     return LIB
 
 

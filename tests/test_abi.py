@@ -101,3 +101,20 @@ def test_variant_b_shapes_rejected_before_launch(lib):
     st = lib.dspark_markov_draft(fake, fake, fake, 1, 64, fake, fake, 4, 4, 1024, fake, fake, fake, None,
                                  fake, ws, None)
     assert st == 1
+
+
+def test_probe_library_rejects_bad_arguments():
+    """The benchmark's L2 read probe (its own shared object, outside the
+    library's path) loads without a GPU and rejects bad arguments before any
+    launch."""
+    path = os.path.join(ROOT, "speculative_decoding_semi_b200", "libdspark_probe.so")
+    probe = ctypes.CDLL(path)
+    probe.dspark_probe_l2_read.restype = ctypes.c_int
+    probe.dspark_probe_l2_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_size_t, ctypes.c_void_p]
+    probe.dspark_probe_sink_words.restype = ctypes.c_size_t
+    assert probe.dspark_probe_l2_read(None, 1 << 20, 4, None, 1 << 20, None) == 1
+    assert probe.dspark_probe_l2_read(ctypes.c_void_p(16), 1 << 20, 4, None, 1 << 20, None) == 1
+    assert probe.dspark_probe_l2_read(ctypes.c_void_p(17), 1 << 20, 4, ctypes.c_void_p(64), 1 << 20, None) == 1
+    assert probe.dspark_probe_l2_read(ctypes.c_void_p(16), 24, 4, ctypes.c_void_p(64), 1 << 20, None) == 1
+    assert probe.dspark_probe_l2_read(ctypes.c_void_p(16), 1 << 20, 0, ctypes.c_void_p(64), 1 << 20, None) == 1
