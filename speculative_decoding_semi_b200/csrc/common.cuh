@@ -251,76 +251,6 @@ __device__ __forceinline__ void cta_release_add(unsigned* ctr, unsigned v) {
   }
 }
 
-// One warp: the first element (vocabulary order) of a run of n elements
-// (n a multiple of 4) whose running fp64 sum of weights exceeds R, with a
-// positive weight; -1 if rounding leaves none (*last_pos then gives the last
-// positive one). Elements are read as coalesced rows of 128: lane l holds
-// elements 4l..4l+3 of each row, `load(e)` returns the data for elements
-// e..e+3 and `weigh(data, w)` their four weights. Up to kRows rows are loaded
-// at once into registers before scanning; longer runs go row by row.
-template <int kRows, class T, class Load, class Weigh>
-__device__ __forceinline__ int scan_rows128(int n, int lane, double R, Load load, Weigh weigh, int* last_pos) {
-  const int nrows = (n + 127) / 128;
-  double before = 0.0;
-  int found = -1, last = -1;
-  auto process = [&](int r0, const T& v) {
-    const int e = r0 + 4 * lane;
-    double w[4] = {0.0, 0.0, 0.0, 0.0};
-    if (e < n) weigh(v, w);
-    const double ls = ((w[0] + w[1]) + w[2]) + w[3];
-    double inc = ls;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double nb = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += nb;
-    }
-    double exc = __shfl_up_sync(0xffffffffu, inc, 1);
-    if (lane == 0) exc = 0.0;
-    const double ex_l = before + exc;
-    int hitc = -1;
-    if (e < n && ex_l + ls > R) {
-      double cc = ex_l;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (hitc < 0 && cc + w[c] > R && w[c] > 0.0) hitc = c;
-        cc += w[c];
-      }
-    }
-    const unsigned hits = __ballot_sync(0xffffffffu, hitc >= 0);
-    if (hits) {
-      const int hl = __ffs(hits) - 1;
-      found = r0 + 4 * hl + __shfl_sync(0xffffffffu, hitc, hl);
-    }
-    int lp = -1;
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      if (e + c < n && w[c] > 0.0) lp = e + c;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lp = max(lp, __shfl_xor_sync(0xffffffffu, lp, o));
-    last = max(last, lp);
-    before += __shfl_sync(0xffffffffu, inc, 31);
-  };
-  if (nrows <= kRows) {
-    T buf[kRows];
-#pragma unroll
-    for (int j = 0; j < kRows; ++j) {
-      const int e = j * 128 + 4 * lane;
-      if (j < nrows && e < n) buf[j] = load(e);
-    }
-#pragma unroll
-    for (int j = 0; j < kRows; ++j)
-      if (j < nrows && found < 0) process(j * 128, buf[j]);
-  } else {
-    for (int r0 = 0; r0 < n && found < 0; r0 += 128) {
-      T v;
-      if (r0 + 4 * lane < n) v = load(r0 + 4 * lane);
-      process(r0, v);
-    }
-  }
-  *last_pos = last;
-  return found;
-}
-
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
   return __uint_as_float(static_cast<unsigned>(b) << 16);
 }
@@ -416,39 +346,6 @@ __device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
   return r;
 }
 
-// TwoSum of two pairs: s = fl(a + b) and the exact rounding error e, a + b = s + e.
-__device__ __forceinline__ void two_sum2(F2 a, F2 b, F2* s, F2* e) {
-  *s = add2(a, b);
-  const F2 bv = sub2(*s, a);
-  *e = add2(sub2(a, sub2(*s, bv)), sub2(b, bv));
-}
-
-// exp_fine of two values at once: the fp32 steps in pairs, the table lookup,
-// exponent scaling and final fp64 FMA per value (same arithmetic, same result).
-__device__ __forceinline__ void exp_fine2(F2 zh, F2 zl, const double* t16, double* w0, double* w1) {
-  const F2 kInvC = f2(23.083120654223414f, 23.083120654223414f);
-  const F2 kMagic = f2(12582912.f, 12582912.f);
-  const F2 kNC1 = f2(-0.0433349609375f, -0.0433349609375f);
-  const F2 kNC2 = f2(1.326215250341961e-05f, 1.326215250341961e-05f);
-  const F2 x = f2(fmin_nan(fmax_nan(f2_lo(zh), -708.f), 709.f), fmin_nan(fmax_nan(f2_hi(zh), -708.f), 709.f));
-  const F2 tn = fma2(x, kInvC, kMagic);
-  const F2 n = sub2(tn, kMagic);
-  F2 r = fma2(n, kNC1, x);
-  r = fma2(n, kNC2, r);
-  r = add2(r, zl);
-  F2 q = fma2(r, f2(1.f / 120.f, 1.f / 120.f), f2(1.f / 24.f, 1.f / 24.f));
-  q = fma2(q, r, f2(1.f / 6.f, 1.f / 6.f));
-  q = fma2(q, r, f2(0.5f, 0.5f));
-  q = fma2(q, r, f2(1.f, 1.f));
-  const F2 p = mul2(q, r);
-  const int n0 = __float_as_int(f2_lo(tn)) - 0x4B400000, n1 = __float_as_int(f2_hi(tn)) - 0x4B400000;
-  const double t0 = t16[n0 & 15], t1 = t16[n1 & 15];
-  const double s0 = __hiloint2double(__double2hiint(t0) + (n0 >> 4) * (1 << 20), __double2loint(t0));
-  const double s1 = __hiloint2double(__double2hiint(t1) + (n1 >> 4) * (1 << 20), __double2loint(t1));
-  *w0 = fma(s0, static_cast<double>(f2_lo(p)), s0);
-  *w1 = fma(s1, static_cast<double>(f2_hi(p)), s1);
-}
-
 // e^(x + y) for two pairs, where zh = fl(x + y) is already formed: the same
 // table-driven steps as exp_fine, with the reduced argument built from x and y
 // themselves, r = (x - n ln2/16) + y, so that the rounding error of zh never
@@ -498,12 +395,6 @@ __device__ __forceinline__ double warp_transpose_sum16(double (&v)[16], int lane
     }
   }
   return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
-}
-
-// fp32 -> bf16 bits, round to nearest even (finite inputs).
-__device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
-  const unsigned u = __float_as_uint(x);
-  return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
 }
 
 }  // namespace dspark
