@@ -23,7 +23,9 @@ teacher forcing); forced acceptance counts that fix which row the final token
 comes from; zero Markov factors reduce the draft to independent per-position
 inverse-CDF sampling; the bias equals a brute-force fp64 triple loop; the
 scheduler equals brute force over every length assignment; survival has
-closed forms at c=0 and c -> +-inf.
+closed forms at c=0 and c -> +-inf; a request sample, packed target rows and
+a vanished residual (fallback to p) agree with the full batch, the dense
+layout and a scipy draw from p.
 """
 from __future__ import annotations
 
